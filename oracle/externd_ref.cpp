@@ -1,0 +1,461 @@
+// ExTernD CPU oracle -- TEST INFRASTRUCTURE ONLY.
+//
+// A plain, slow, single-threaded statement of the expanded-rank ternary
+// decomposition, used only by the tests, by the package's smoke check and by
+// the benchmark's CPU-baseline leg to check and time the CUDA path.  The CUDA
+// library never links, loads or calls this file, and this file shares no code
+// with it.
+//
+// Sources (web pages on arXiv:2607.13511, "ExTernD: Expanded-Rank Ternary
+// Decomposition"):
+//   [REV]  "Paper Review: ExTernD ..." (romaanj.github.io), sections "Method"
+//          and "Key idea".
+//   [PITH] "Pith review of ExTernD ..." (pith.science), "What carries the
+//          argument", the referee report (paper Sec. 2.3 greedy ALS,
+//          Sec. 2.4 block-ALS with Eq. 3, Sec. 2.5 importance weighting,
+//          Appendix A Prop. 1 and Prop. 2) and "Assumptions & free
+//          parameters" (Eq. 2 threshold, Eq. 5 packing).
+//   [ABS]  the paper's abstract as reprinted on arxivlens.com.
+//
+// Readings taken where the pages leave a step open (each is listed in the
+// design notes with its reason):
+//   * T_tau(x)_j = sign(x_j) if |x_j| > tau * rms(x) else 0; rms over the
+//     whole vector, computed in fp64; strict comparison.
+//   * The residual R is kept in the input's precision (fp32).  A deflation
+//     R_ij <- R_ij - u_i v_j d is one IEEE fp32 add or subtract of the fp32
+//     scale d (u_i v_j is +-1 or 0), never fused with anything else.
+//   * Every other reduction (matrix-vector products, norms, scales) is fp64.
+//   * Ties in every argmax go to the lowest (row-major) index.
+//   * Weighted mode: the u-step thresholds y = R (w o v); the v-step
+//     thresholds z = R^T u unweighted (per-column weights do not move the
+//     column-wise least-squares minimiser); d = u^T R W v / (|u|^2 v^T W v).
+//   * The single-entry safeguard scores entries by w_j R_ij^2; in weighted
+//     mode that score is formed in fp32 as (R_ij * R_ij) * w_j so that the
+//     argmax is decided in the same precision as the kernel's.
+//   * Block mode: eps = 1e-6 * trace(G) / b for each b x b Gram system G
+//     (1.0 when the trace is zero); U-step target R W V (V^T W V + eps I)^-1;
+//     V-step target ((U^T U + eps I)^-1 U^T R)^T (Eq. 3); joint scales
+//     D = (G + eps I)^-1 r with G = (U^T U) o (V^T W V), r_l = u_l^T R W v_l;
+//     b ordered rank-1 deflations; no safeguard.
+//
+// Build: g++ -O2 -ffp-contract=off -fno-fast-math -shared -fPIC (see build.py).
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+namespace {
+
+inline double wt(const float* w, int64_t j) { return w ? (double)w[j] : 1.0; }
+
+// Cholesky factorisation and solve of a small symmetric positive definite
+// system, fp64, in place.  Returns false if a pivot is not positive.
+bool chol_solve(std::vector<double>& G, int64_t b, std::vector<double>& rhs, int64_t nrhs) {
+  // G is b x b row-major; rhs is b x nrhs row-major.
+  for (int64_t i = 0; i < b; ++i) {
+    for (int64_t j = 0; j <= i; ++j) {
+      double s = G[i * b + j];
+      for (int64_t p = 0; p < j; ++p) s -= G[i * b + p] * G[j * b + p];
+      if (i == j) {
+        if (!(s > 0.0)) return false;
+        G[i * b + i] = std::sqrt(s);
+      } else {
+        G[i * b + j] = s / G[j * b + j];
+      }
+    }
+  }
+  for (int64_t c = 0; c < nrhs; ++c) {
+    for (int64_t i = 0; i < b; ++i) {  // L y = r
+      double s = rhs[i * nrhs + c];
+      for (int64_t p = 0; p < i; ++p) s -= G[i * b + p] * rhs[p * nrhs + c];
+      rhs[i * nrhs + c] = s / G[i * b + i];
+    }
+    for (int64_t i = b - 1; i >= 0; --i) {  // L^T x = y
+      double s = rhs[i * nrhs + c];
+      for (int64_t p = i + 1; p < b; ++p) s -= G[p * b + i] * rhs[p * nrhs + c];
+      rhs[i * nrhs + c] = s / G[i * b + i];
+    }
+  }
+  return true;
+}
+
+double ridge_eps(const std::vector<double>& G, int64_t b) {
+  double tr = 0.0;
+  for (int64_t i = 0; i < b; ++i) tr += G[i * b + i];
+  return tr > 0.0 ? 1e-6 * tr / (double)b : 1.0;
+}
+
+}  // namespace
+
+extern "C" {
+
+// T_tau, the adaptive ternarisation operator ([PITH] Eq. 2 via "Assumptions &
+// free parameters"; [REV] "Method": tau sets the share of zeros).  Writes the
+// ternary codes and returns the threshold tau * rms(x).
+double orc_ternarize(const double* x, int64_t len, double tau, int8_t* out) {
+  double s = 0.0;
+  for (int64_t j = 0; j < len; ++j) s += x[j] * x[j];
+  double thr = len > 0 ? tau * std::sqrt(s / (double)len) : 0.0;
+  for (int64_t j = 0; j < len; ++j) {
+    double a = std::fabs(x[j]);
+    out[j] = (a > thr) ? (x[j] > 0.0 ? 1 : -1) : 0;
+  }
+  return thr;
+}
+
+// ALS u half-step ([PITH] referee summary, Sec. 2.3: ternarise against the
+// current residual): y = R (w o v), u = T_tau(y).  Returns the threshold.
+double orc_u_step(const float* R, int64_t m, int64_t n, const int8_t* v, const float* w,
+                  double tau, double* y, int8_t* u) {
+  for (int64_t i = 0; i < m; ++i) {
+    double s = 0.0;
+    const float* row = R + i * n;
+    for (int64_t j = 0; j < n; ++j)
+      if (v[j]) s += (double)row[j] * ((double)v[j] * wt(w, j));
+    y[i] = s;
+  }
+  return orc_ternarize(y, m, tau, u);
+}
+
+// ALS v half-step: z = R^T u, v = T_tau(z).  Returns the threshold.
+double orc_v_step(const float* R, int64_t m, int64_t n, const int8_t* u, double tau,
+                  double* z, int8_t* v) {
+  for (int64_t j = 0; j < n; ++j) z[j] = 0.0;
+  for (int64_t i = 0; i < m; ++i) {
+    if (!u[i]) continue;
+    const float* row = R + i * n;
+    for (int64_t j = 0; j < n; ++j) z[j] += (double)u[i] * (double)row[j];
+  }
+  return orc_ternarize(z, n, tau, v);
+}
+
+// Row energies rho_i = sum_j w_j R_ij^2; returns the index of the largest
+// (lowest index on ties).  The component's starting row.
+int64_t orc_row_norms(const float* R, int64_t m, int64_t n, const float* w, double* rho) {
+  int64_t best = 0;
+  for (int64_t i = 0; i < m; ++i) {
+    double s = 0.0;
+    const float* row = R + i * n;
+    for (int64_t j = 0; j < n; ++j) s += wt(w, j) * (double)row[j] * (double)row[j];
+    rho[i] = s;
+    if (s > rho[best]) best = i;
+  }
+  return best;
+}
+
+// Weighted squared Frobenius norm sum_ij w_j R_ij^2 (energy, [PITH]
+// "Load-bearing premise": E = 1 - |A - Ahat|^2 / |A|^2).
+double orc_sumsq(const float* R, int64_t m, int64_t n, const float* w) {
+  double s = 0.0;
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t j = 0; j < n; ++j) s += wt(w, j) * (double)R[i * n + j] * (double)R[i * n + j];
+  return s;
+}
+
+// Best single entry for the safeguard ([PITH] referee major comment 1,
+// Appendix A Prop. 2): argmax of w_j R_ij^2, lowest row-major index on ties.
+// Writes the score M (as fp64) and returns the flat index.
+int64_t orc_entry_max(const float* R, int64_t m, int64_t n, const float* w, double* M) {
+  int64_t best = 0;
+  if (w) {
+    float bs = -1.0f;
+    for (int64_t i = 0; i < m; ++i)
+      for (int64_t j = 0; j < n; ++j) {
+        float r = R[i * n + j];
+        float sq = r * r;
+        float s = sq * w[j];
+        if (s > bs) { bs = s; best = i * n + j; }
+      }
+    *M = (double)bs;
+  } else {
+    float ba = -1.0f;
+    for (int64_t i = 0; i < m; ++i)
+      for (int64_t j = 0; j < n; ++j) {
+        float a = std::fabs(R[i * n + j]);
+        if (a > ba) { ba = a; best = i * n + j; }
+      }
+    *M = (double)ba * (double)ba;
+  }
+  return best;
+}
+
+// Closed-form scale and gain ([PITH] "What carries the argument": d = u^T R v /
+// (|u|^2 |v|^2); Prop. 1: the residual falls by (u^T R v)^2 / (|u|^2 |v|^2)).
+// z must be R^T u for the given u; then u^T R W v = sum_j w_j v_j z_j.
+// out[0]=p=u^T R W v, out[1]=n_u, out[2]=n_v, out[3]=|u|^2 v^T W v,
+// out[4]=d (exact fp64), out[5]=gain.
+void orc_scale(const double* z, const int8_t* u, const int8_t* v, int64_t m, int64_t n,
+               const float* w, double* out) {
+  double p = 0.0, vw = 0.0;
+  int64_t nu = 0, nv = 0;
+  for (int64_t i = 0; i < m; ++i) nu += u[i] != 0;
+  for (int64_t j = 0; j < n; ++j)
+    if (v[j]) {
+      ++nv;
+      p += wt(w, j) * (double)v[j] * z[j];
+      vw += wt(w, j);
+    }
+  double den = (double)nu * vw;
+  out[0] = p;
+  out[1] = (double)nu;
+  out[2] = (double)nv;
+  out[3] = den;
+  out[4] = den > 0.0 ? p / den : 0.0;
+  out[5] = den > 0.0 ? p * p / den : 0.0;
+}
+
+// Rank-1 deflation R <- R - d u v^T ([REV] "Method": deflate the residual
+// before the next component), one fp32 add or subtract per touched entry.
+void orc_deflate(float* R, int64_t m, int64_t n, const int8_t* u, const int8_t* v, float d) {
+  for (int64_t i = 0; i < m; ++i) {
+    if (!u[i]) continue;
+    float* row = R + i * n;
+    for (int64_t j = 0; j < n; ++j) {
+      int s = (int)u[i] * (int)v[j];
+      if (s > 0) row[j] = row[j] - d;
+      else if (s < 0) row[j] = row[j] + d;
+    }
+  }
+}
+
+// Greedy sequential-deflation ALS (paper Sec. 2.3 per [PITH]; [REV] "Method"
+// and "Key idea"), with the best-single-entry safeguard of Prop. 2.
+// Outputs: U k x m and V k x n ternary codes (row c = component c), D[k],
+// energy[k] = 1 - |R_{c+1}|_W^2 / |A|_W^2, init_row[k] (row whose ternarised
+// copy started the component), fallback[k] (1 when the safeguard fired).
+// Returns the number of safeguard activations.
+int64_t orc_decompose_seq(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                          const float* w, int8_t* U, int8_t* V, float* D, double* energy,
+                          int64_t* init_row, uint8_t* fallback) {
+  std::vector<float> R(A, A + m * n);
+  std::vector<double> rho(m), y(m), z(n), rowd(n);
+  std::vector<int8_t> u(m), v(n);
+  const double E0 = orc_sumsq(A, m, n, w);
+  int64_t nfb = 0;
+  bool zero = false;
+  for (int64_t c = 0; c < k; ++c) {
+    int8_t* Uc = U + c * m;
+    int8_t* Vc = V + c * n;
+    if (!zero) {
+      double M = 0.0;
+      int64_t flat = orc_entry_max(R.data(), m, n, w, &M);
+      if (M == 0.0) zero = true;
+      if (!zero) {
+        int64_t istar = orc_row_norms(R.data(), m, n, w, rho.data());
+        init_row[c] = istar;
+        for (int64_t j = 0; j < n; ++j) rowd[j] = (double)R[istar * n + j];
+        orc_ternarize(rowd.data(), n, tau, v.data());
+        for (int t = 0; t < iters; ++t) {
+          orc_u_step(R.data(), m, n, v.data(), w, tau, y.data(), u.data());
+          orc_v_step(R.data(), m, n, u.data(), tau, z.data(), v.data());
+        }
+        double sc[6];
+        orc_scale(z.data(), u.data(), v.data(), m, n, w, sc);
+        float d;
+        if (sc[5] < M) {  // safeguard: single best entry removal
+          std::fill(u.begin(), u.end(), 0);
+          std::fill(v.begin(), v.end(), 0);
+          int64_t ip = flat / n, jp = flat % n;
+          u[ip] = 1;
+          v[jp] = 1;
+          d = R[flat];
+          fallback[c] = 1;
+          ++nfb;
+        } else {
+          d = (float)sc[4];
+          fallback[c] = 0;
+        }
+        orc_deflate(R.data(), m, n, u.data(), v.data(), d);
+        std::memcpy(Uc, u.data(), m);
+        std::memcpy(Vc, v.data(), n);
+        D[c] = d;
+        energy[c] = E0 > 0.0 ? 1.0 - orc_sumsq(R.data(), m, n, w) / E0 : 1.0;
+        continue;
+      }
+    }
+    // R is identically zero: the remaining components are empty.
+    std::memset(Uc, 0, m);
+    std::memset(Vc, 0, n);
+    D[c] = 0.0f;
+    energy[c] = 1.0;
+    init_row[c] = -1;
+    fallback[c] = 0;
+  }
+  return nfb;
+}
+
+// Replays components [0, upto) onto A with the same fp32 deflation; the
+// residual R_upto it yields is the one component `upto` started from.
+void orc_replay(const float* A, int64_t m, int64_t n, const int8_t* U, const int8_t* V,
+                const float* D, int64_t upto, float* R) {
+  std::memcpy(R, A, sizeof(float) * m * n);
+  for (int64_t c = 0; c < upto; ++c) orc_deflate(R, m, n, U + c * m, V + c * n, D[c]);
+}
+
+// Ahat = B diag(D) C in fp64 ([ABS]: A ~ B diag(D) C).
+void orc_reconstruct(const int8_t* U, const int8_t* V, const float* D, int64_t m, int64_t n,
+                     int64_t k, double* Ahat) {
+  std::memset(Ahat, 0, sizeof(double) * m * n);
+  for (int64_t c = 0; c < k; ++c) {
+    const int8_t* u = U + c * m;
+    const int8_t* v = V + c * n;
+    double d = D[c];
+    for (int64_t i = 0; i < m; ++i) {
+      if (!u[i]) continue;
+      for (int64_t j = 0; j < n; ++j)
+        if (v[j]) Ahat[i * n + j] += d * (double)(u[i] * v[j]);
+    }
+  }
+}
+
+// Indices of the b largest row energies, distinct, descending, lowest index
+// first on ties (block-ALS initialisation).
+void orc_top_rows(const double* rho, int64_t m, int64_t b, int64_t* rows) {
+  std::vector<int64_t> idx(m);
+  for (int64_t i = 0; i < m; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(),
+                   [&](int64_t a, int64_t c) { return rho[a] > rho[c]; });
+  for (int64_t l = 0; l < b; ++l) rows[l] = idx[l];
+}
+
+// Block-ALS with decorrelated least-squares targets (paper Sec. 2.4, Eq. 3 per
+// [PITH]; [REV] "Method": batched block-ALS).  Fits bb = min(b, k - c0)
+// components per sweep.  Outputs as orc_decompose_seq; energy per component
+// from the closed form |R|^2 - 2 sum d_l r_l + sum d_l d_l' G_ll' over the
+// block prefix.
+void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                         const float* w, int64_t b, int8_t* U, int8_t* V, float* D,
+                         double* energy, int64_t* init_row) {
+  std::vector<float> R(A, A + m * n);
+  const double E0 = orc_sumsq(A, m, n, w);
+  std::vector<double> rho(m);
+  for (int64_t c0 = 0; c0 < k; c0 += b) {
+    const int64_t bb = std::min(b, k - c0);
+    orc_row_norms(R.data(), m, n, w, rho.data());
+    std::vector<int64_t> rows(bb);
+    orc_top_rows(rho.data(), m, bb, rows.data());
+    std::vector<int8_t> Ub(m * bb, 0), Vb(n * bb, 0);  // column l of U is Ub[i*bb+l]
+    std::vector<double> col(std::max(m, n));
+    std::vector<int8_t> code(std::max(m, n));
+    for (int64_t l = 0; l < bb; ++l) {
+      init_row[c0 + l] = rows[l];
+      for (int64_t j = 0; j < n; ++j) col[j] = (double)R[rows[l] * n + j];
+      orc_ternarize(col.data(), n, tau, code.data());
+      for (int64_t j = 0; j < n; ++j) Vb[j * bb + l] = code[j];
+    }
+    std::vector<double> G(bb * bb), P, Q;
+    for (int t = 0; t < iters; ++t) {
+      // U-step: P = R W V, target P (V^T W V + eps I)^-1, threshold per column.
+      for (int64_t l = 0; l < bb; ++l)
+        for (int64_t l2 = 0; l2 < bb; ++l2) {
+          double s = 0.0;
+          for (int64_t j = 0; j < n; ++j) s += wt(w, j) * Vb[j * bb + l] * Vb[j * bb + l2];
+          G[l * bb + l2] = s;
+        }
+      double eps = ridge_eps(G, bb);
+      for (int64_t l = 0; l < bb; ++l) G[l * bb + l] += eps;
+      P.assign(m * bb, 0.0);
+      for (int64_t i = 0; i < m; ++i)
+        for (int64_t l = 0; l < bb; ++l) {
+          double s = 0.0;
+          for (int64_t j = 0; j < n; ++j)
+            if (Vb[j * bb + l]) s += (double)R[i * n + j] * wt(w, j) * Vb[j * bb + l];
+          P[i * bb + l] = s;
+        }
+      // rows of P^T solved against the symmetric system: T = P G^-1 <=> G T^T = P^T
+      std::vector<double> Pt(bb * m);
+      for (int64_t i = 0; i < m; ++i)
+        for (int64_t l = 0; l < bb; ++l) Pt[l * m + i] = P[i * bb + l];
+      std::vector<double> Gc = G;
+      chol_solve(Gc, bb, Pt, m);
+      for (int64_t l = 0; l < bb; ++l) {
+        orc_ternarize(&Pt[l * m], m, tau, code.data());
+        for (int64_t i = 0; i < m; ++i) Ub[i * bb + l] = code[i];
+      }
+      // V-step (Eq. 3): V = T_col(((U^T U + eps I)^-1 U^T R)^T).
+      for (int64_t l = 0; l < bb; ++l)
+        for (int64_t l2 = 0; l2 < bb; ++l2) {
+          double s = 0.0;
+          for (int64_t i = 0; i < m; ++i) s += (double)(Ub[i * bb + l] * Ub[i * bb + l2]);
+          G[l * bb + l2] = s;
+        }
+      eps = ridge_eps(G, bb);
+      for (int64_t l = 0; l < bb; ++l) G[l * bb + l] += eps;
+      Q.assign(bb * n, 0.0);
+      for (int64_t l = 0; l < bb; ++l)
+        for (int64_t i = 0; i < m; ++i) {
+          int8_t ui = Ub[i * bb + l];
+          if (!ui) continue;
+          for (int64_t j = 0; j < n; ++j) Q[l * n + j] += (double)ui * (double)R[i * n + j];
+        }
+      Gc = G;
+      chol_solve(Gc, bb, Q, n);
+      for (int64_t l = 0; l < bb; ++l) {
+        orc_ternarize(&Q[l * n], n, tau, code.data());
+        for (int64_t j = 0; j < n; ++j) Vb[j * bb + l] = code[j];
+      }
+    }
+    // Joint scales: (G + eps I) D = r with G = (U^T U) o (V^T W V).
+    std::vector<double> GU(bb * bb), GV(bb * bb), r(bb, 0.0);
+    for (int64_t l = 0; l < bb; ++l)
+      for (int64_t l2 = 0; l2 < bb; ++l2) {
+        double su = 0.0, sv = 0.0;
+        for (int64_t i = 0; i < m; ++i) su += (double)(Ub[i * bb + l] * Ub[i * bb + l2]);
+        for (int64_t j = 0; j < n; ++j) sv += wt(w, j) * Vb[j * bb + l] * Vb[j * bb + l2];
+        GU[l * bb + l2] = su;
+        GV[l * bb + l2] = sv;
+      }
+    for (int64_t l = 0; l < bb; ++l) {
+      double s = 0.0;
+      for (int64_t i = 0; i < m; ++i) {
+        int8_t ui = Ub[i * bb + l];
+        if (!ui) continue;
+        for (int64_t j = 0; j < n; ++j)
+          if (Vb[j * bb + l]) s += (double)ui * (double)R[i * n + j] * wt(w, j) * Vb[j * bb + l];
+      }
+      r[l] = s;
+    }
+    for (int64_t l = 0; l < bb; ++l)
+      for (int64_t l2 = 0; l2 < bb; ++l2) G[l * bb + l2] = GU[l * bb + l2] * GV[l * bb + l2];
+    std::vector<double> Graw = G;
+    double eps = ridge_eps(G, bb);
+    // components with an empty u or v take d = 0 and drop out of the system
+    std::vector<int64_t> act;
+    for (int64_t l = 0; l < bb; ++l)
+      if (GU[l * bb + l] > 0.0 && GV[l * bb + l] > 0.0) act.push_back(l);
+    std::vector<double> dsol(bb, 0.0);
+    if (!act.empty()) {
+      int64_t na = (int64_t)act.size();
+      std::vector<double> Ga(na * na), ra(na);
+      for (int64_t a = 0; a < na; ++a) {
+        ra[a] = r[act[a]];
+        for (int64_t c = 0; c < na; ++c) Ga[a * na + c] = G[act[a] * bb + act[c]];
+        Ga[a * na + a] += eps;
+      }
+      chol_solve(Ga, na, ra, 1);
+      for (int64_t a = 0; a < na; ++a) dsol[act[a]] = ra[a];
+    }
+    std::vector<float> dl(bb);
+    for (int64_t l = 0; l < bb; ++l) dl[l] = (float)dsol[l];
+    double base = orc_sumsq(R.data(), m, n, w);
+    std::vector<int8_t> uc(m), vc(n);
+    for (int64_t l = 0; l < bb; ++l) {
+      for (int64_t i = 0; i < m; ++i) uc[i] = Ub[i * bb + l];
+      for (int64_t j = 0; j < n; ++j) vc[j] = Vb[j * bb + l];
+      orc_deflate(R.data(), m, n, uc.data(), vc.data(), dl[l]);
+      std::memcpy(U + (c0 + l) * m, uc.data(), m);
+      std::memcpy(V + (c0 + l) * n, vc.data(), n);
+      D[c0 + l] = dl[l];
+      double e = base;
+      for (int64_t a = 0; a <= l; ++a) {
+        e -= 2.0 * (double)dl[a] * r[a];
+        for (int64_t c = 0; c <= l; ++c) e += (double)dl[a] * (double)dl[c] * Graw[a * bb + c];
+      }
+      energy[c0 + l] = E0 > 0.0 ? 1.0 - e / E0 : 1.0;
+    }
+  }
+}
+
+}  // extern "C"

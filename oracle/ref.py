@@ -1,0 +1,201 @@
+"""Python view of the ExTernD CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+Thin numpy/ctypes marshalling over ``externd_ref.cpp``.  Only the tests, the
+package's smoke check and the benchmark's CPU-baseline leg import this
+module; the CUDA library never does.  Codes are int8 in {-1, 0, +1}; U is
+k x m and V is k x n (row c holds component c), so B = U^T and C = V.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_F = ctypes.POINTER(ctypes.c_float)
+_D = ctypes.POINTER(ctypes.c_double)
+_I8 = ctypes.POINTER(ctypes.c_int8)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
+_I64 = ctypes.POINTER(ctypes.c_int64)
+_i64 = ctypes.c_int64
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(_build.build())
+        L.orc_ternarize.argtypes = [_D, _i64, ctypes.c_double, _I8]
+        L.orc_ternarize.restype = ctypes.c_double
+        L.orc_u_step.argtypes = [_F, _i64, _i64, _I8, _F, ctypes.c_double, _D, _I8]
+        L.orc_u_step.restype = ctypes.c_double
+        L.orc_v_step.argtypes = [_F, _i64, _i64, _I8, ctypes.c_double, _D, _I8]
+        L.orc_v_step.restype = ctypes.c_double
+        L.orc_row_norms.argtypes = [_F, _i64, _i64, _F, _D]
+        L.orc_row_norms.restype = _i64
+        L.orc_sumsq.argtypes = [_F, _i64, _i64, _F]
+        L.orc_sumsq.restype = ctypes.c_double
+        L.orc_entry_max.argtypes = [_F, _i64, _i64, _F, _D]
+        L.orc_entry_max.restype = _i64
+        L.orc_scale.argtypes = [_D, _I8, _I8, _i64, _i64, _F, _D]
+        L.orc_scale.restype = None
+        L.orc_deflate.argtypes = [_F, _i64, _i64, _I8, _I8, ctypes.c_float]
+        L.orc_deflate.restype = None
+        L.orc_decompose_seq.argtypes = [_F, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _F,
+                                        _I8, _I8, _F, _D, _I64, _U8]
+        L.orc_decompose_seq.restype = _i64
+        L.orc_replay.argtypes = [_F, _i64, _i64, _I8, _I8, _F, _i64, _F]
+        L.orc_replay.restype = None
+        L.orc_reconstruct.argtypes = [_I8, _I8, _F, _i64, _i64, _i64, _D]
+        L.orc_reconstruct.restype = None
+        L.orc_top_rows.argtypes = [_D, _i64, _i64, _I64]
+        L.orc_top_rows.restype = None
+        L.orc_decompose_block.argtypes = [_F, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _F,
+                                          _i64, _I8, _I8, _F, _D, _I64]
+        L.orc_decompose_block.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a: Optional[np.ndarray], t):
+    if a is None:
+        return ctypes.cast(None, t)
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(t)
+
+
+def _f32(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+
+def ternarize(x: np.ndarray, tau: float):
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape[0], np.int8)
+    thr = lib().orc_ternarize(_p(x, _D), x.shape[0], tau, _p(out, _I8))
+    return out, thr
+
+
+def u_step(R: np.ndarray, v: np.ndarray, tau: float, w=None):
+    R = _f32(R); w = _f32(w)
+    m, n = R.shape
+    v = np.ascontiguousarray(v, np.int8)
+    y = np.empty(m); u = np.empty(m, np.int8)
+    thr = lib().orc_u_step(_p(R, _F), m, n, _p(v, _I8), _p(w, _F), tau, _p(y, _D), _p(u, _I8))
+    return u, y, thr
+
+
+def v_step(R: np.ndarray, u: np.ndarray, tau: float):
+    R = _f32(R)
+    m, n = R.shape
+    u = np.ascontiguousarray(u, np.int8)
+    z = np.empty(n); v = np.empty(n, np.int8)
+    thr = lib().orc_v_step(_p(R, _F), m, n, _p(u, _I8), tau, _p(z, _D), _p(v, _I8))
+    return v, z, thr
+
+
+def row_norms(R, w=None):
+    R = _f32(R); w = _f32(w)
+    m, n = R.shape
+    rho = np.empty(m)
+    best = lib().orc_row_norms(_p(R, _F), m, n, _p(w, _F), _p(rho, _D))
+    return rho, int(best)
+
+
+def sumsq(R, w=None):
+    R = _f32(R); w = _f32(w)
+    return float(lib().orc_sumsq(_p(R, _F), R.shape[0], R.shape[1], _p(w, _F)))
+
+
+def entry_max(R, w=None):
+    R = _f32(R); w = _f32(w)
+    M = ctypes.c_double()
+    flat = lib().orc_entry_max(_p(R, _F), R.shape[0], R.shape[1], _p(w, _F), ctypes.byref(M))
+    return int(flat), float(M.value)
+
+
+@dataclass
+class Scale:
+    p: float
+    n_u: int
+    n_v: int
+    den: float
+    d: float
+    gain: float
+
+
+def scale(z, u, v, w=None) -> Scale:
+    z = np.ascontiguousarray(z, np.float64)
+    u = np.ascontiguousarray(u, np.int8); v = np.ascontiguousarray(v, np.int8)
+    w = _f32(w)
+    out = np.empty(6)
+    lib().orc_scale(_p(z, _D), _p(u, _I8), _p(v, _I8), u.shape[0], v.shape[0], _p(w, _F),
+                    _p(out, _D))
+    return Scale(out[0], int(out[1]), int(out[2]), out[3], out[4], out[5])
+
+
+def deflate(R: np.ndarray, u, v, d: float) -> np.ndarray:
+    """Returns a deflated copy of R."""
+    R = np.array(R, dtype=np.float32, order="C", copy=True)
+    u = np.ascontiguousarray(u, np.int8); v = np.ascontiguousarray(v, np.int8)
+    lib().orc_deflate(_p(R, _F), R.shape[0], R.shape[1], _p(u, _I8), _p(v, _I8),
+                      ctypes.c_float(np.float32(d)))
+    return R
+
+
+@dataclass
+class Decomposition:
+    U: np.ndarray         # k x m int8 (B^T)
+    V: np.ndarray         # k x n int8 (C)
+    D: np.ndarray         # k fp32
+    energy: np.ndarray    # k fp64
+    init_row: np.ndarray  # k int64
+    fallback: np.ndarray  # k uint8 (sequential mode only)
+    n_fallback: int
+
+
+def decompose(A, k: int, tau: float, iters: int, w=None, block: int = 1,
+              block_path: bool = False) -> Decomposition:
+    """Free-running decomposition; block > 1 (or block_path) runs block-ALS."""
+    A = _f32(A); w = _f32(w)
+    m, n = A.shape
+    U = np.zeros((k, m), np.int8); V = np.zeros((k, n), np.int8)
+    D = np.zeros(k, np.float32); E = np.zeros(k); rows = np.zeros(k, np.int64)
+    fb = np.zeros(k, np.uint8)
+    if block <= 1 and not block_path:
+        nfb = lib().orc_decompose_seq(_p(A, _F), m, n, k, tau, iters, _p(w, _F), _p(U, _I8),
+                                      _p(V, _I8), _p(D, _F), _p(E, _D), _p(rows, _I64),
+                                      _p(fb, _U8))
+    else:
+        lib().orc_decompose_block(_p(A, _F), m, n, k, tau, iters, _p(w, _F), block, _p(U, _I8),
+                                  _p(V, _I8), _p(D, _F), _p(E, _D), _p(rows, _I64))
+        nfb = 0
+    return Decomposition(U, V, D, E, rows, fb, int(nfb))
+
+
+def replay(A, U, V, D, upto: int) -> np.ndarray:
+    A = _f32(A)
+    m, n = A.shape
+    R = np.empty_like(A)
+    U = np.ascontiguousarray(U, np.int8); V = np.ascontiguousarray(V, np.int8)
+    D = _f32(D)
+    lib().orc_replay(_p(A, _F), m, n, _p(U, _I8), _p(V, _I8), _p(D, _F), upto, _p(R, _F))
+    return R
+
+
+def reconstruct(U, V, D, m: int, n: int) -> np.ndarray:
+    U = np.ascontiguousarray(U, np.int8); V = np.ascontiguousarray(V, np.int8)
+    D = _f32(D)
+    out = np.empty((m, n))
+    lib().orc_reconstruct(_p(U, _I8), _p(V, _I8), _p(D, _F), m, n, D.shape[0], _p(out, _D))
+    return out
+
+
+def top_rows(rho, b: int):
+    rho = np.ascontiguousarray(rho, np.float64)
+    rows = np.empty(b, np.int64)
+    lib().orc_top_rows(_p(rho, _D), rho.shape[0], b, _p(rows, _I64))
+    return rows
