@@ -1,0 +1,48 @@
+// Internal interfaces between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace externd {
+
+struct SeqHostArgs {
+  const float* A;
+  int64_t m, n, k;
+  float tau;
+  int iters;
+  const float* w;
+  uint32_t* packed_B;
+  uint32_t* packed_C;
+  float* D;
+  double* energy;
+  int64_t ntrace;
+  const int64_t* trace_comp;
+  uint32_t* trace_bits;
+  int32_t* trace_row;
+  uint8_t* trace_flags;
+  int64_t* stats;
+  int64_t wait_budget;
+};
+
+struct BlockHostArgs {
+  const float* A;
+  int64_t m, n, k;
+  float tau;
+  int iters;
+  const float* w;
+  int block;
+  uint32_t* packed_B;
+  uint32_t* packed_C;
+  float* D;
+  double* energy;
+  int64_t* stats;
+};
+
+int seq_decompose(const SeqHostArgs& h, cudaStream_t st);
+int block_decompose(const BlockHostArgs& h, cudaStream_t st);
+int reconstruct(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
+                int64_t k, float* out, cudaStream_t st);
+int* status_word_ptr();
+
+}  // namespace externd

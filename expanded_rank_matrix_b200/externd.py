@@ -1,0 +1,225 @@
+"""ctypes binding to libexternd.so (the C ABI in include/externd.h).
+
+Argument marshalling only: every step of the decomposition runs in the CUDA
+library.  PyTorch supplies device memory and streams.  There is no fallback:
+if the library is missing or no CUDA device is present the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libexternd.so")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_CUDA = -2
+ERR_OOM = -3
+ERR_NO_COOP = -4
+ERR_TIMEOUT = -5
+ERR_NONFINITE = -6
+
+# every symbol include/externd.h declares
+EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_traced",
+           "externd_reconstruct", "externd_sync_status")
+
+_lib = None
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+class ExterndError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed with status {code}")
+        self.code = code
+
+
+def load(path: str = LIB_PATH):
+    """Loads the library (no GPU needed) and declares the signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libexternd.so is not built ({path}); run __graft_entry__.build()")
+    L = ctypes.CDLL(path)
+    L.externd_rank.argtypes = [_i64, _i64, ctypes.c_float]
+    L.externd_rank.restype = _i64
+    L.externd_decompose.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float, ctypes.c_int,
+                                    _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
+    L.externd_decompose.restype = ctypes.c_int
+    L.externd_decompose_traced.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
+                                           ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                           _i64, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
+    L.externd_decompose_traced.restype = ctypes.c_int
+    L.externd_reconstruct.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]
+    L.externd_reconstruct.restype = ctypes.c_int
+    L.externd_sync_status.argtypes = [_vp]
+    L.externd_sync_status.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def rank(m: int, n: int, mu: float) -> int:
+    return int(load().externd_rank(m, n, mu))
+
+
+def words(length: int) -> int:
+    return (length + 31) // 32
+
+
+@dataclass
+class Factors:
+    """Device-resident result of one decomposition."""
+    packed_B: torch.Tensor  # int32 view of uint32 [k, 2, ceil(m/32)]
+    packed_C: torch.Tensor  # [k, 2, ceil(n/32)]
+    D: torch.Tensor         # fp32 [k]
+    energy: torch.Tensor    # fp64 [k]
+    m: int
+    n: int
+
+    @property
+    def k(self) -> int:
+        return int(self.D.shape[0])
+
+
+def alloc_factors(m: int, n: int, k: int, device) -> Factors:
+    return Factors(torch.empty((k, 2, words(m)), dtype=torch.int32, device=device),
+                   torch.empty((k, 2, words(n)), dtype=torch.int32, device=device),
+                   torch.empty(k, dtype=torch.float32, device=device),
+                   torch.empty(k, dtype=torch.float64, device=device), m, n)
+
+
+def decompose_into(out: Factors, A: torch.Tensor, mu: float, tau: float, iters: int,
+                   w: Optional[torch.Tensor] = None, block: int = 1,
+                   stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Runs externd_decompose into preallocated outputs (stream ordered)."""
+    m, n = A.shape
+    rc = load().externd_decompose(_ptr(A), m, n, mu, tau, iters, _ptr(w), block,
+                                  _ptr(out.packed_B), _ptr(out.packed_C), _ptr(out.D),
+                                  _ptr(out.energy), _stream(stream))
+    if rc != OK:
+        raise ExterndError(rc, "externd_decompose")
+
+
+def decompose(A: torch.Tensor, mu: float, tau: float, iters: int,
+              w: Optional[torch.Tensor] = None, block: int = 1,
+              stream: Optional[torch.cuda.Stream] = None, check: bool = True) -> Factors:
+    if A.dtype != torch.float32 or A.dim() != 2:
+        raise ValueError("A must be a 2-D fp32 CUDA tensor")
+    m, n = A.shape
+    k = rank(m, n, mu)
+    if k < 1:
+        raise ExterndError(ERR_INVALID_ARG, "externd_rank")
+    out = alloc_factors(m, n, k, A.device)
+    decompose_into(out, A, mu, tau, iters, w, block, stream)
+    if check:
+        st = sync_status(stream)
+        if st != OK:
+            raise ExterndError(st, "externd_decompose (device)")
+    return out
+
+
+@dataclass
+class Trace:
+    comps: np.ndarray   # traced component indices
+    bits: torch.Tensor  # [ntrace, S] int32
+    row: torch.Tensor   # [ntrace] int32
+    flags: torch.Tensor  # [ntrace] uint8
+    stats: torch.Tensor  # [4] int64
+    iters: int
+
+
+def decompose_traced(A: torch.Tensor, mu: float, tau: float, iters: int,
+                     trace_comps: Sequence[int], w: Optional[torch.Tensor] = None,
+                     wait_budget: int = 0, stream: Optional[torch.cuda.Stream] = None,
+                     check: bool = True):
+    m, n = A.shape
+    k = rank(m, n, mu)
+    out = alloc_factors(m, n, k, A.device)
+    comps = np.array(sorted(set(int(c) for c in trace_comps if 0 <= c < k)), dtype=np.int64)
+    nt = int(comps.size)
+    S = 2 * words(n) + iters * 2 * (words(m) + words(n))
+    dev = A.device
+    tc = torch.from_numpy(comps).to(dev) if nt else None
+    tb = torch.zeros((max(nt, 1), S), dtype=torch.int32, device=dev)
+    tr = torch.zeros(max(nt, 1), dtype=torch.int32, device=dev)
+    tf = torch.zeros(max(nt, 1), dtype=torch.uint8, device=dev)
+    stats = torch.zeros(4, dtype=torch.int64, device=dev)
+    rc = load().externd_decompose_traced(
+        _ptr(A), m, n, mu, tau, iters, _ptr(w), 1, _ptr(out.packed_B), _ptr(out.packed_C),
+        _ptr(out.D), _ptr(out.energy), nt, _ptr(tc), _ptr(tb) if nt else None,
+        _ptr(tr) if nt else None, _ptr(tf) if nt else None, _ptr(stats), wait_budget,
+        _stream(stream))
+    if rc != OK:
+        raise ExterndError(rc, "externd_decompose_traced")
+    status = sync_status(stream)
+    if check and status != OK:
+        raise ExterndError(status, "externd_decompose_traced (device)")
+    return out, Trace(comps, tb[:nt], tr[:nt], tf[:nt], stats, iters), status
+
+
+def reconstruct(f: Factors, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    out = torch.empty((f.m, f.n), dtype=torch.float32, device=f.D.device)
+    rc = load().externd_reconstruct(_ptr(f.packed_B), _ptr(f.packed_C), _ptr(f.D), f.m, f.n, f.k,
+                                    _ptr(out), _stream(stream))
+    if rc != OK:
+        raise ExterndError(rc, "externd_reconstruct")
+    return out
+
+
+def sync_status(stream: Optional[torch.cuda.Stream] = None) -> int:
+    return int(load().externd_sync_status(_stream(stream)))
+
+
+# --- decoding of packed outputs (host side, for inspection and tests) -------
+
+def unpack_planes(packed: np.ndarray, length: int) -> np.ndarray:
+    """[..., 2, W] uint32 bitplanes -> [..., length] int8 codes in {-1,0,1}."""
+    p = np.ascontiguousarray(packed).view(np.uint32)
+    bits = ((p[..., :, :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.int8)
+    bits = bits.reshape(*p.shape[:-1], -1)[..., :length]
+    mask, sign = bits[..., 0, :], bits[..., 1, :]
+    return (mask * (1 - 2 * sign)).astype(np.int8)
+
+
+def to_codes(f: Factors):
+    """(U k x m, V k x n, D, energy) on the host."""
+    U = unpack_planes(f.packed_B.cpu().numpy(), f.m)
+    V = unpack_planes(f.packed_C.cpu().numpy(), f.n)
+    return U, V, f.D.cpu().numpy(), f.energy.cpu().numpy()
+
+
+def trace_vectors(tr: Trace, t_idx: int, m: int, n: int):
+    """Decodes traced component t_idx into (v0, [u_1..u_I], [v_1..v_I])."""
+    Wm, Wn = words(m), words(n)
+    b = tr.bits[t_idx].cpu().numpy().view(np.uint32)
+    v0 = unpack_planes(b[:2 * Wn].reshape(2, Wn), n)
+    us, vs = [], []
+    off = 2 * Wn
+    for _ in range(tr.iters):
+        us.append(unpack_planes(b[off:off + 2 * Wm].reshape(2, Wm), m))
+        off += 2 * Wm
+        vs.append(unpack_planes(b[off:off + 2 * Wn].reshape(2, Wn), n))
+        off += 2 * Wn
+    return v0, us, vs

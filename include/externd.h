@@ -1,0 +1,147 @@
+/*
+ * externd.h -- C ABI of libexternd.so, the B200 (sm_100a) ExTernD library.
+ *
+ * ExTernD ("Expanded-Rank Ternary Decomposition", arXiv:2607.13511) factors
+ * an fp32 matrix A (m x n) as A ~ B diag(D) C with ternary B in
+ * {-1,0,+1}^{m x k}, ternary C in {-1,0,+1}^{k x n}, real D in R^k and an
+ * inner rank k = floor(mu * min(m, n)) that may exceed min(m, n)
+ * (the paper's abstract; "Method" in the romaanj.github.io review).
+ *
+ * Conventions shared by every entry point:
+ *  - Every array pointer is a caller-owned DEVICE pointer on the current CUDA
+ *    device, at least 4-byte aligned.  The library never frees or keeps them.
+ *  - Matrices are row-major (C order); A[i*n + j] is row i, column j.
+ *  - Packed ternary vectors ("bitplanes", mask+sign as in the paper's Eq. 5
+ *    bit accounting): a vector of length L is 2 planes of W = ceil(L/32)
+ *    uint32 words.  Bit b of word t stands for entry 32*t + b.  Plane 0 is the
+ *    mask (1 = nonzero), plane 1 the sign (1 = -1).  The sign bit is 0
+ *    wherever the mask bit is 0, and bits past L are 0, so packed outputs can
+ *    be compared bit for bit.
+ *      packed_B: k x 2 x ceil(m/32) words -- component c's column of B.
+ *      packed_C: k x 2 x ceil(n/32) words -- component c's row of C.
+ *  - Calls are ordered on `stream`.  The return value reports errors found on
+ *    the host (arguments, allocation, launch).  Errors found on the device
+ *    (a wait that ran out, non-finite input) go to a per-device status word
+ *    that externd_sync_status() returns.
+ *  - Scratch memory is taken with cudaMallocAsync on `stream` and released on
+ *    `stream` before the call returns.
+ */
+#ifndef EXTERND_H
+#define EXTERND_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+#define EXTERND_OK 0
+#define EXTERND_ERR_INVALID_ARG (-1) /* bad size, pointer, alignment or knob   */
+#define EXTERND_ERR_CUDA (-2)        /* a CUDA runtime call failed              */
+#define EXTERND_ERR_OOM (-3)         /* scratch allocation failed               */
+#define EXTERND_ERR_NO_COOP (-4)     /* the persistent grid cannot be resident  */
+#define EXTERND_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out      */
+#define EXTERND_ERR_NONFINITE (-6)   /* NaN/Inf in A, or w not finite and > 0   */
+
+typedef struct CUstream_st* externd_stream_t; /* same object as cudaStream_t */
+
+/*
+ * externd_rank -- the inner rank k = floor(mu * min(m, n)) (the paper's
+ * abstract: k = mu min(m, n)).  Returns 0 when an argument is out of range.
+ */
+int64_t externd_rank(int64_t m, int64_t n, float mu);
+
+/*
+ * externd_decompose -- the whole ExTernD decomposition of one matrix.
+ *
+ * block == 1: greedy sequential-deflation ALS (paper Sec. 2.3, per the Pith
+ *   review's referee summary and the review's "Method"/"Key idea"): for each
+ *   component c = 0..k-1 on the residual R (R = A at the start):
+ *     i*  = argmax_i sum_j w_j R_ij^2;  v = T_tau(R[i*, :])
+ *     repeat iters times: u = T_tau(R W v); v = T_tau(R^T u)
+ *     d = u^T R W v / (|u|^2 v^T W v), gain g = (u^T R W v)^2 / (|u|^2 v^T W v)
+ *     if g < max_ij w_j R_ij^2: u = e_i', v = e_j', d = R_i'j' (single-entry
+ *       safeguard of Appendix A, Prop. 2)
+ *     R <- R - d u v^T  (one fp32 add or subtract per touched entry)
+ *   where T_tau(x)_j = sign(x_j) if |x_j| > tau * rms(x) else 0 (Eq. 2) and
+ *   W = diag(w) (W = I when w is NULL; the importance weighting of Sec. 2.5).
+ * block > 1: block-ALS (Sec. 2.4, Eq. 3): b = block components per sweep
+ *   against decorrelated least-squares targets, joint scales, b ordered
+ *   rank-1 deflations.
+ *
+ * Arguments:
+ *   A            [m*n] fp32, read only.
+ *   m, n         1 <= m, n and m*n < 2^31.
+ *   mu           rank multiplier, > 0; k = externd_rank(m, n, mu) >= 1.
+ *   tau          threshold factor, finite and >= 0.
+ *   iters        ALS iterations per component (or per block), >= 1.
+ *   w            [n] fp32 per-input-column importance weights, finite and
+ *                > 0, or NULL for the unweighted objective.
+ *   block        1 (sequential) or 2..min(k, 256) (block-ALS).
+ *   packed_B     [k][2][ceil(m/32)] uint32 out.
+ *   packed_C     [k][2][ceil(n/32)] uint32 out.
+ *   D            [k] fp32 out.
+ *   energy_trace [k] fp64 out: 1 - |R_{c+1}|_W^2 / |A|_W^2 after component c
+ *                (|X|_W^2 = sum_ij w_j X_ij^2; 1 when A == 0).
+ *   stream       CUDA stream (NULL = legacy default stream).
+ * Returns EXTERND_OK or a negative status.  On a device-detected error the
+ * outputs are undefined and externd_sync_status() returns the error.
+ */
+int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
+                      const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
+                      float* D, double* energy_trace, externd_stream_t stream);
+
+/*
+ * externd_decompose_traced -- externd_decompose plus a record of the ALS
+ * trajectory of selected components (used to compare the device path with a
+ * reference half-step by half-step).  Sequential mode (block == 1) only.
+ *
+ *   trace_comp   [ntrace] int64, strictly increasing component indices, or
+ *                NULL when ntrace == 0.
+ *   trace_bits   [ntrace][S] uint32 out, S = 2*Wn + iters*2*(Wm + Wn),
+ *                Wm = ceil(m/32), Wn = ceil(n/32): for each traced component
+ *                the packed starting v, then for t = 1..iters the packed u_t
+ *                and the packed v_t.  May be NULL when ntrace == 0.
+ *   trace_row    [ntrace] int32 out: the starting row i*.
+ *   trace_flags  [ntrace] uint8 out: bit 0 = the safeguard replaced the ALS
+ *                pair of this component.
+ *   stats        [4] int64 out or NULL: [0] safeguard activations over all
+ *                components, [1] components emitted as zero because the
+ *                residual vanished, [2] launch clusters, [3] CTAs per cluster.
+ *   wait_budget  upper bound, in SM clock cycles, on every device-side wait
+ *                for another CTA's data; 0 selects the default (about 1 s).
+ *                A wait that runs out sets EXTERND_ERR_TIMEOUT and the kernel
+ *                winds down without further waits.
+ */
+int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
+                             const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
+                             float* D, double* energy_trace, int64_t ntrace,
+                             const int64_t* trace_comp, uint32_t* trace_bits, int32_t* trace_row,
+                             uint8_t* trace_flags, int64_t* stats, int64_t wait_budget,
+                             externd_stream_t stream);
+
+/*
+ * externd_reconstruct -- A_hat = B diag(D) C from the packed factors (the
+ * factor form of the paper's abstract), accumulated in fp64 in component
+ * order and rounded once to fp32.
+ *   packed_B [k][2][ceil(m/32)], packed_C [k][2][ceil(n/32)], D [k] in;
+ *   A_hat [m*n] fp32 out.  1 <= m, n, k; m*n < 2^31.
+ */
+int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, const float* D,
+                        int64_t m, int64_t n, int64_t k, float* A_hat, externd_stream_t stream);
+
+/*
+ * externd_sync_status -- synchronises `stream`, then returns and clears the
+ * current device's status word: EXTERND_OK, or the first device-side error
+ * (EXTERND_ERR_TIMEOUT, EXTERND_ERR_NONFINITE) raised by any call on this
+ * device since the last read; EXTERND_ERR_CUDA if the synchronisation
+ * itself failed.
+ */
+int externd_sync_status(externd_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXTERND_H */

@@ -294,6 +294,12 @@ void orc_replay(const float* A, int64_t m, int64_t n, const int8_t* U, const int
   for (int64_t c = 0; c < upto; ++c) orc_deflate(R, m, n, U + c * m, V + c * n, D[c]);
 }
 
+// In-place replay of components [from, to) onto R (R must hold R_from).
+void orc_replay_range(float* R, int64_t m, int64_t n, const int8_t* U, const int8_t* V,
+                      const float* D, int64_t from, int64_t to) {
+  for (int64_t c = from; c < to; ++c) orc_deflate(R, m, n, U + c * m, V + c * n, D[c]);
+}
+
 // Ahat = B diag(D) C in fp64 ([ABS]: A ~ B diag(D) C).
 void orc_reconstruct(const int8_t* U, const int8_t* V, const float* D, int64_t m, int64_t n,
                      int64_t k, double* Ahat) {

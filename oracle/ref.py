@@ -50,6 +50,8 @@ def lib():
         L.orc_decompose_seq.restype = _i64
         L.orc_replay.argtypes = [_F, _i64, _i64, _I8, _I8, _F, _i64, _F]
         L.orc_replay.restype = None
+        L.orc_replay_range.argtypes = [_F, _i64, _i64, _I8, _I8, _F, _i64, _i64]
+        L.orc_replay_range.restype = None
         L.orc_reconstruct.argtypes = [_I8, _I8, _F, _i64, _i64, _i64, _D]
         L.orc_reconstruct.restype = None
         L.orc_top_rows.argtypes = [_D, _i64, _i64, _I64]
@@ -184,6 +186,15 @@ def replay(A, U, V, D, upto: int) -> np.ndarray:
     D = _f32(D)
     lib().orc_replay(_p(A, _F), m, n, _p(U, _I8), _p(V, _I8), _p(D, _F), upto, _p(R, _F))
     return R
+
+
+def replay_range(R: np.ndarray, U, V, D, start: int, stop: int) -> None:
+    """Deflates R in place by components [start, stop)."""
+    assert R.dtype == np.float32 and R.flags["C_CONTIGUOUS"]
+    U = np.ascontiguousarray(U, np.int8); V = np.ascontiguousarray(V, np.int8)
+    D = _f32(D)
+    lib().orc_replay_range(_p(R, _F), R.shape[0], R.shape[1], _p(U, _I8), _p(V, _I8), _p(D, _F),
+                           start, stop)
 
 
 def reconstruct(U, V, D, m: int, n: int) -> np.ndarray:

@@ -1,0 +1,111 @@
+"""Teacher-forced comparison of the CUDA path with the CPU oracle.
+
+The oracle rebuilds the device's residual R_c exactly by replaying the
+device's emitted (u, v, d) components onto A with the same fp32 deflation,
+then re-runs each traced half-step from the device's own input iterate:
+  v0  = T_tau(R_c[i*, :])          from the device's starting row i*
+  u_t = T_tau(R_c W v_{t-1})       from the device's v_{t-1}
+  v_t = T_tau(R_c^T u_t)           from the device's u_t
+and checks every ternary code bit for bit, except codes whose |x_j| lies
+within BAND (relative) of the threshold tau * rms(x); those are counted and
+reported, not hidden.  Scales agree to D_RTOL relative, residual norms to
+NORM_RTOL relative.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+BAND = 1e-5
+D_RTOL = 1e-5
+NORM_RTOL = 1e-5
+
+
+@dataclass
+class Report:
+    comps: int = 0
+    codes: int = 0
+    band_total: int = 0
+    band_mismatch: int = 0
+    bad: list = field(default_factory=list)
+    fallbacks: int = 0
+    init_ties: int = 0
+
+    def fail(self, msg):
+        if len(self.bad) < 20:
+            self.bad.append(msg)
+
+    @property
+    def ok(self) -> bool:
+        return not self.bad
+
+
+def _cmp(rep: Report, tag: str, gpu: np.ndarray, ora: np.ndarray, x: np.ndarray, thr: float):
+    band = np.abs(np.abs(x) - thr) <= BAND * max(thr, 1e-300)
+    mism = gpu != ora
+    rep.codes += gpu.size
+    rep.band_total += int(band.sum())
+    rep.band_mismatch += int((mism & band).sum())
+    hard = mism & ~band
+    if hard.any():
+        idx = np.flatnonzero(hard)[:5]
+        rep.fail(f"{tag}: {int(hard.sum())} codes differ outside the band, e.g. at {idx.tolist()} "
+                 f"x={x[idx].tolist()} thr={thr}")
+
+
+def check_component(oracle, rep: Report, c: int, R: np.ndarray, E0: float, tau: float, iters: int,
+                    w, trace_row: int, v0: np.ndarray, us, vs, flag: int, U_c: np.ndarray,
+                    V_c: np.ndarray, D_c: float, energy_c: float) -> np.ndarray:
+    """Checks component c given R = R_c; returns R_{c+1} (replayed with the
+    device's emitted component)."""
+    rep.comps += 1
+    rho, best = oracle.row_norms(R, w)
+    i0 = int(trace_row)
+    if not (0 <= i0 < R.shape[0]) or rho[i0] < rho.max() * (1 - 1e-5):
+        rep.fail(f"comp {c}: start row {i0} is not a largest-energy row (best {best})")
+        return oracle.deflate(R, U_c, V_c, D_c)
+    if i0 != best:
+        rep.init_ties += 1
+    row = R[i0].astype(np.float64)
+    v0o, thr0 = oracle.ternarize(row, tau)
+    _cmp(rep, f"comp {c} v0", v0, v0o, row, thr0)
+    vprev = v0
+    z = None
+    for t in range(iters):
+        uo, y, thr = oracle.u_step(R, vprev, tau, w)
+        _cmp(rep, f"comp {c} u{t + 1}", us[t], uo, y, thr)
+        vo, z, thr2 = oracle.v_step(R, us[t], tau)
+        _cmp(rep, f"comp {c} v{t + 1}", vs[t], vo, z, thr2)
+        vprev = vs[t]
+    s = oracle.scale(z, us[-1], vs[-1], w)
+    flat, M = oracle.entry_max(R, w)
+    fb_o = s.gain < M
+    close = abs(s.gain - M) <= 1e-5 * max(M, 1e-300)
+    if bool(flag) != fb_o and not close:
+        rep.fail(f"comp {c}: safeguard decision differs (gain {s.gain}, M {M}, device {flag})")
+    if flag:
+        rep.fallbacks += 1
+        i = int(np.flatnonzero(U_c)[0]) if U_c.any() else -1
+        j = int(np.flatnonzero(V_c)[0]) if V_c.any() else -1
+        if i < 0 or j < 0 or np.count_nonzero(U_c) != 1 or np.count_nonzero(V_c) != 1:
+            rep.fail(f"comp {c}: safeguard component is not a single entry")
+        else:
+            wj = 1.0 if w is None else float(w[j])
+            sc = float(np.float32(np.float32(R[i, j] * R[i, j]) * np.float32(wj))) if w is not None \
+                else float(R[i, j]) ** 2
+            if sc < M * (1 - 1e-6):
+                rep.fail(f"comp {c}: safeguard entry ({i},{j}) is not a largest entry")
+            if np.float32(D_c) != R[i, j]:
+                rep.fail(f"comp {c}: safeguard scale {D_c} != R_ij {R[i, j]}")
+    else:
+        if not (np.array_equal(U_c, us[-1]) and np.array_equal(V_c, vs[-1])):
+            rep.fail(f"comp {c}: emitted factors differ from the last iterates")
+        if abs(float(D_c) - s.d) > D_RTOL * abs(s.d) + 1e-30:
+            rep.fail(f"comp {c}: scale {D_c} vs oracle {s.d}")
+    Rn = oracle.deflate(R, U_c, V_c, D_c)
+    res_o = oracle.sumsq(Rn, w)
+    res_g = (1.0 - float(energy_c)) * E0
+    if abs(res_g - res_o) > NORM_RTOL * res_o + 1e-12 * E0:
+        rep.fail(f"comp {c}: residual |R|^2 {res_g} vs oracle {res_o}")
+    return Rn

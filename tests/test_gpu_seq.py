@@ -1,0 +1,170 @@
+"""Parity of the CUDA sequential-deflation path (block = 1) with the CPU
+oracle, through the C ABI.  Needs a B200."""
+import numpy as np
+import pytest
+import torch
+
+from expanded_rank_matrix_b200 import externd as X
+from expanded_rank_matrix_b200 import workloads as W
+from tests.parity import Report, check_component
+
+pytestmark = pytest.mark.gpu
+
+FREE_ENERGY_ATOL = 1e-4
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def teacher_forced(oracle, A, mu, tau, iters, comps=None, w=None):
+    """Runs the traced device path and checks the traced components (all when
+    comps is None).  Returns (report, factors, trace)."""
+    m, n = A.shape
+    k = X.rank(m, n, mu)
+    comps = list(range(k)) if comps is None else sorted(set(comps))
+    f, tr, status = X.decompose_traced(_dev(A), mu, tau, iters, comps,
+                                       w=None if w is None else _dev(w))
+    assert status == X.OK
+    U, V, D, E = X.to_codes(f)
+    rows = tr.row.cpu().numpy()
+    flags = tr.flags.cpu().numpy()
+    E0 = oracle.sumsq(A, w)
+    rep = Report()
+    R = np.array(A, dtype=np.float32, copy=True)
+    at = 0
+    for ti, c in enumerate(tr.comps.tolist()):
+        oracle.replay_range(R, U, V, D, at, c)
+        v0, us, vs = X.trace_vectors(tr, ti, m, n)
+        R = check_component(oracle, rep, c, R, E0, tau, iters, w, rows[ti], v0, us, vs, flags[ti],
+                            U[c], V[c], D[c], E[c])
+        at = c + 1
+    return rep, f, tr
+
+
+def test_iid256_teacher_forced_every_component(oracle):
+    wl = W.config_small()
+    rep, f, tr = teacher_forced(oracle, wl.a, wl.mu, wl.tau, wl.iters)
+    print(f"iid256: {rep.comps} comps, {rep.codes} codes, band {rep.band_total} "
+          f"(mismatch {rep.band_mismatch}), fallbacks {rep.fallbacks}, init ties {rep.init_ties}")
+    assert rep.ok, rep.bad
+    assert rep.comps == wl.k
+
+
+def test_iid256_free_running_energy(oracle):
+    wl = W.config_small()
+    f = X.decompose(_dev(wl.a), wl.mu, wl.tau, wl.iters)
+    E = f.energy.cpu().numpy()
+    ref = oracle.decompose(wl.a, wl.k, wl.tau, wl.iters)
+    assert abs(E[-1] - ref.energy[-1]) <= FREE_ENERGY_ATOL
+    # energy after every component stays close along the whole trajectory
+    assert np.max(np.abs(E - ref.energy)) <= 5e-3
+    assert np.all(np.diff(E) >= -4 * 2.0 ** -24)
+
+
+def test_reconstruct_bit_exact_against_oracle(oracle):
+    wl = W.config_small()
+    f = X.decompose(_dev(wl.a), wl.mu, wl.tau, wl.iters)
+    Ahat = X.reconstruct(f).cpu().numpy()
+    U, V, D, E = X.to_codes(f)
+    ref = oracle.reconstruct(U, V, D, wl.m, wl.n).astype(np.float32)
+    assert np.array_equal(Ahat.view(np.uint32), ref.view(np.uint32))
+    A64 = wl.a.astype(np.float64)
+    e = 1.0 - ((A64 - Ahat) ** 2).sum() / (A64 ** 2).sum()
+    assert e == pytest.approx(E[-1], abs=1e-5)
+
+
+def test_deterministic_and_prefix_consistent():
+    wl = W.config_small()
+    A = _dev(wl.a)
+    f1 = X.decompose(A, 2.0, wl.tau, wl.iters)
+    f2 = X.decompose(A, 2.0, wl.tau, wl.iters)
+    f3 = X.decompose(A, 1.0, wl.tau, wl.iters)
+    for a, b in ((f1.packed_B, f2.packed_B), (f1.packed_C, f2.packed_C), (f1.D, f2.D),
+                 (f1.energy, f2.energy)):
+        assert torch.equal(a, b)
+    k = f3.k
+    assert torch.equal(f1.packed_B[:k], f3.packed_B) and torch.equal(f1.packed_C[:k], f3.packed_C)
+    assert torch.equal(f1.D[:k], f3.D) and torch.equal(f1.energy[:k], f3.energy)
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (2, 2), (3, 3), (1, 70), (70, 1), (37, 53), (33, 65),
+                                   (130, 97), (257, 300)])
+def test_edge_shapes_teacher_forced(oracle, shape):
+    m, n = shape
+    A = W.iid_gaussian(m, n, 1000 + m * 7 + n)
+    mu = 2.0 if min(m, n) > 1 else 3.0
+    rep, f, tr = teacher_forced(oracle, A, mu, 0.5, 3)
+    assert rep.ok, rep.bad
+    ref = oracle.decompose(A, f.k, 0.5, 3)
+    assert abs(float(f.energy[-1]) - ref.energy[-1]) <= FREE_ENERGY_ATOL
+
+
+def test_weighted_teacher_forced(oracle):
+    A = W.llm_like(192, 160, 77, n_outliers=4)
+    w = W.lognormal_weights(160, 77)
+    rep, f, tr = teacher_forced(oracle, A, 2.0, 0.5, 4, w=w)
+    print(f"weighted 192x160: band {rep.band_total} mismatch {rep.band_mismatch} "
+          f"fallbacks {rep.fallbacks}")
+    assert rep.ok, rep.bad
+    ref = oracle.decompose(A, f.k, 0.5, 4, w=w)
+    assert abs(float(f.energy[-1]) - ref.energy[-1]) <= FREE_ENERGY_ATOL
+
+
+def test_unit_weights_match_unweighted():
+    A = _dev(W.llm_like(128, 96, 5, n_outliers=2))
+    f0 = X.decompose(A, 2.0, 0.5, 4)
+    f1 = X.decompose(A, 2.0, 0.5, 4, w=torch.ones(96, device="cuda"))
+    assert torch.equal(f0.packed_B, f1.packed_B) and torch.equal(f0.packed_C, f1.packed_C)
+    assert torch.equal(f0.D, f1.D)
+
+
+def test_safeguard_path(oracle):
+    # tau so large that every ALS pair is empty: every component is the
+    # single-entry step, which must zero the chosen entry exactly.
+    A = W.iid_gaussian(64, 48, 8)
+    rep, f, tr = teacher_forced(oracle, A, 1.0, 50.0, 2)
+    assert rep.ok, rep.bad
+    assert rep.fallbacks == f.k
+    assert int(tr.stats[0]) == f.k
+
+
+def test_zero_matrix():
+    A = torch.zeros((96, 80), device="cuda")
+    f = X.decompose(A, 2.0, 0.5, 3)
+    assert not f.packed_B.any() and not f.packed_C.any() and not f.D.any()
+    assert torch.all(f.energy == 1.0)
+
+
+def test_nonfinite_input_reports_status():
+    A = torch.randn((64, 64), device="cuda")
+    A[3, 5] = float("nan")
+    with pytest.raises(X.ExterndError) as e:
+        X.decompose(A, 1.0, 0.5, 2)
+    assert e.value.code == X.ERR_NONFINITE
+    w = torch.ones(64, device="cuda")
+    w[7] = -1.0
+    with pytest.raises(X.ExterndError) as e:
+        X.decompose(torch.randn((64, 64), device="cuda"), 1.0, 0.5, 2, w=w)
+    assert e.value.code == X.ERR_NONFINITE
+
+
+def test_wait_budget_runs_out_cleanly():
+    # a one-cycle budget makes the cross-CTA waits give up: the call must end
+    # with EXTERND_ERR_TIMEOUT and leave the context usable
+    A = _dev(W.llm_like(512, 512, 9))
+    f, tr, status = X.decompose_traced(A, 1.0, 0.5, 2, [], wait_budget=1, check=False)
+    assert status in (X.ERR_TIMEOUT, X.OK)
+    f2 = X.decompose(A, 1.0, 0.5, 2)
+    assert X.sync_status() == X.OK
+    assert float(f2.energy[-1]) > 0.5
+
+
+def test_invalid_arguments():
+    A = torch.randn((16, 16), device="cuda")
+    for kw in (dict(mu=0.0), dict(tau=-1.0), dict(iters=0), dict(tau=float("inf"))):
+        args = dict(mu=1.0, tau=0.5, iters=2)
+        args.update(kw)
+        with pytest.raises(X.ExterndError) as e:
+            X.decompose(A, **args)
+        assert e.value.code == X.ERR_INVALID_ARG
