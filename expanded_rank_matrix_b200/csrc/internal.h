@@ -44,5 +44,7 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st);
 int reconstruct(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
                 int64_t k, float* out, cudaStream_t st);
 int* status_word_ptr();
+int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
+                               cudaStream_t st);
 
 }  // namespace externd

@@ -969,4 +969,60 @@ int seq_decompose(const SeqHostArgs& h, cudaStream_t st) {
   return rc;
 }
 
+
+// Same launch as seq_decompose, but the exchange ring and the abort word live
+// in caller-provided device scratch instead of a cudaMallocAsync workspace,
+// and only plans whose residual tiles stay in shared memory are accepted (a
+// global tile store would need m*n*4 bytes of scratch).  No allocation.
+int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
+                               cudaStream_t st) {
+  SeqPlan pl;
+  cudaError_t e = plan_seq((int)h.m, (int)h.n, st, &pl);
+  if (e == cudaErrorNotSupported) return EXTERND_ERR_NO_COOP;
+  if (e != cudaSuccess) return EXTERND_ERR_CUDA;
+  if (!pl.smt) return EXTERND_ERR_SCRATCH_LIMIT;
+  const int recw = pl.TCp + 16;
+  const long long slot_words = (long long)pl.NC * pl.CS * recw;
+  const size_t xbytes = sizeof(uint64_t) * 3 * (size_t)slot_words;
+  const size_t abort_off = (xbytes + 255) & ~(size_t)255;
+  const size_t need = abort_off + 256;
+  if (need > scratch_bytes) return EXTERND_ERR_SCRATCH_LIMIT;
+  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return EXTERND_ERR_CUDA;
+  SeqArgs a = {};
+  a.A = h.A;
+  a.m = (int)h.m;
+  a.n = (int)h.n;
+  a.k = (int)h.k;
+  a.tau = h.tau;
+  a.iters = h.iters;
+  a.w = h.w;
+  a.pB = h.packed_B;
+  a.pC = h.packed_C;
+  a.D = h.D;
+  a.energy = h.energy;
+  a.NC = pl.NC;
+  a.CS = pl.CS;
+  a.nchr = (a.m + 31) / 32;
+  a.nchc = (a.n + 31) / 32;
+  a.TRmax = pl.TRmax;
+  a.TCp = pl.TCp;
+  a.recw = recw;
+  a.gtile = nullptr;
+  a.xbuf = (uint64_t*)scratch;
+  a.slot_words = slot_words;
+  a.trace_comp = nullptr;
+  a.ntrace = 0;
+  a.budget = kDefaultWaitBudget;
+  a.abort_word = (int*)((char*)scratch + abort_off);
+  a.dev_status = status_word_ptr();
+  if (!a.dev_status) return EXTERND_ERR_CUDA;
+  int dummy = 0;
+  e = dispatch<true>(pl.NQL, a, pl.smem, st, &dummy, false);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return EXTERND_ERR_CUDA;
+  }
+  return EXTERND_OK;
+}
+
 }  // namespace externd

@@ -24,10 +24,11 @@ ERR_OOM = -3
 ERR_NO_COOP = -4
 ERR_TIMEOUT = -5
 ERR_NONFINITE = -6
+ERR_SCRATCH_LIMIT = -7
 
 # every symbol include/externd.h declares
 EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_traced",
-           "externd_reconstruct", "externd_sync_status")
+           "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -59,6 +60,9 @@ def load(path: str = LIB_PATH):
     L.externd_decompose_traced.restype = ctypes.c_int
     L.externd_reconstruct.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]
     L.externd_reconstruct.restype = ctypes.c_int
+    L.externd_decompose_noalloc.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
+                                            ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp]
+    L.externd_decompose_noalloc.restype = ctypes.c_int
     L.externd_sync_status.argtypes = [_vp]
     L.externd_sync_status.restype = ctypes.c_int
     _lib = L
@@ -138,6 +142,17 @@ def decompose(A: torch.Tensor, mu: float, tau: float, iters: int,
         if st != OK:
             raise ExterndError(st, "externd_decompose (device)")
     return out
+
+
+def decompose_noalloc_into(out: Factors, A: torch.Tensor, mu: float, tau: float, iters: int,
+                           w: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None) -> int:
+    """externd_decompose_noalloc into preallocated outputs; returns the C
+    status (the entry point allocates nothing itself)."""
+    m, n = A.shape
+    return int(load().externd_decompose_noalloc(_ptr(A), m, n, mu, tau, iters, _ptr(w),
+                                                _ptr(out.packed_B), _ptr(out.packed_C),
+                                                _ptr(out.D), _ptr(out.energy), _stream(stream)))
 
 
 @dataclass

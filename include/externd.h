@@ -43,6 +43,7 @@ extern "C" {
 #define EXTERND_ERR_NO_COOP (-4)     /* the persistent grid cannot be resident  */
 #define EXTERND_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out      */
 #define EXTERND_ERR_NONFINITE (-6)   /* NaN/Inf in A, or w not finite and > 0   */
+#define EXTERND_ERR_SCRATCH_LIMIT (-7) /* problem too large for the fixed scratch  */
 
 typedef struct CUstream_st* externd_stream_t; /* same object as cudaStream_t */
 
@@ -130,6 +131,41 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
  */
 int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, const float* D,
                         int64_t m, int64_t n, int64_t k, float* A_hat, externd_stream_t stream);
+
+/*
+ * externd_decompose_noalloc -- externd_decompose (block == 1 only) without
+ * any memory allocation.  The paper has no counterpart; this is a service of
+ * this library.
+ *
+ * Some callers cannot let a library allocate device memory: programs whose
+ * memory manager has already reserved the device's memory (a framework's
+ * caching allocator, a serving process that sizes its pools at start-up), in
+ * which a library's own allocation can fail or fragment what they hold; and
+ * latency-bound request paths that forbid allocation after start-up because
+ * allocation calls can stall or synchronise the device.  This entry point
+ * takes all of its scratch (the cross-CTA exchange ring and the abort word)
+ * from one fixed array compiled into the library, EXTERND_NOALLOC_SCRATCH_BYTES
+ * bytes per device, which every device that loads the library holds until the
+ * process exits.  It calls no cudaMalloc, cudaMallocAsync, cudaFree or other
+ * allocating routine.  The caller still owns and passes every input and
+ * output, with the same meaning as for externd_decompose.
+ *
+ * Limits: the residual must fit in the persistent grid's shared memory
+ * (about 26 MB of fp32 on a B200, e.g. 2560 x 2560) and the exchange ring
+ * must fit in the fixed array; larger problems return
+ * EXTERND_ERR_SCRATCH_LIMIT without launching anything.
+ * The first call on a device looks up the device address of the fixed array
+ * (a one-time set-up per device, done with that device current); make that
+ * first call before any stream capture.
+ * Every call on a device shares the one array and clears the part it uses at
+ * the start of the call.  Calls that overlap on the GPU (issued on different
+ * streams without ordering between them) race on it and give undefined
+ * results; order them on one stream or with events.
+ */
+#define EXTERND_NOALLOC_SCRATCH_BYTES (4u << 20)
+int externd_decompose_noalloc(const float* A, int64_t m, int64_t n, float mu, float tau,
+                              int iters, const float* w, uint32_t* packed_B, uint32_t* packed_C,
+                              float* D, double* energy_trace, externd_stream_t stream);
 
 /*
  * externd_sync_status -- synchronises `stream`, then returns and clears the
