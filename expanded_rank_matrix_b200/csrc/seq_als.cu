@@ -9,19 +9,20 @@
 // R <- R - d u v^T before the next component.
 //
 // Layout.  The grid is NC clusters of CS CTAs, one CTA per SM.  Cluster c
-// owns a band of rows (a run of 32-row chunks), CTA q of the cluster owns a
-// band of columns (a run of 32-column chunks), so every CTA holds one
-// TR x TC tile of the residual -- in shared memory when the whole matrix fits
-// in the grid's shared memory, otherwise in a private global-memory (L2/HBM)
-// region that the CTA streams.  The tile never moves; only vectors do:
+// owns a band of rows, CTA q of the cluster owns a band of columns (a run of
+// 32-column chunks), so every CTA holds one TR x TC tile of the residual --
+// in shared memory when the whole matrix fits in the grid's shared memory,
+// otherwise in a private global-memory (L2/HBM) region that the CTA streams.
+// The tile never moves; only vectors do:
 //  * R W v: partial row sums per CTA, all-gathered inside the cluster through
 //    distributed shared memory; the cluster's sum of y^2 crosses clusters.
 //  * R^T u: partial column sums per cluster cross clusters; each CTA sums the
 //    NC partials of its own columns in a fixed order, so every cluster holds
 //    the same z; sum z^2 is combined inside the cluster.
 // Cross-cluster data moves through flag-tagged 64-bit words (payload +
-// epoch), so the arrival of the data is the synchronisation.  Every wait is
-// bounded; a wait that runs out raises EXTERND_ERR_TIMEOUT and the kernel
+// epoch), so the arrival of the data is the synchronisation; independent
+// words are loaded back to back before any of them is waited on.  Every wait
+// is bounded; a wait that runs out raises EXTERND_ERR_TIMEOUT and the kernel
 // winds down without further waits.  All reductions run in a fixed order,
 // so results are bit-reproducible run to run.
 
@@ -58,7 +59,7 @@ struct SeqArgs {
   uint32_t* pC;
   float* D;
   double* energy;
-  int NC, CS, nchr, nchc;
+  int NC, CS, nchc;
   int TRmax, TCp, recw;
   float* gtile;
   uint64_t* xbuf;
@@ -74,13 +75,30 @@ struct SeqArgs {
   int* dev_status;
 };
 
+// phases timed (SM cycles, CTA 0) into stats[kStatPhase0 + p]
+enum {
+  PH_SETUP = 0,
+  PH_YPASS,
+  PH_YGATHER,
+  PH_YXCHG,
+  PH_ZPASS,
+  PH_ZXCHG,
+  PH_ZSYNC,
+  PH_SCALE,
+  PH_DEFLATE,
+  PH_STATS,
+  PH_N
+};
+constexpr int kStatPhase0 = 6;
+
 // Shared-memory carve-up, identical on host and device.  yfull lives in the
 // zred region: their lifetimes (y gather..threshold, z reduction) are disjoint.
 struct SeqSmem {
   size_t red, ired, cx, misc, xd, xu, tile, uval, ypart, yfull, rho_p, rmax, rmaxv, rmaxj, zred,
       wcol, vval, zfull, nnzu, total;
-  __host__ __device__ SeqSmem(int TRmax, int TCp, int NC, bool smem_tile) {
+  __host__ __device__ SeqSmem(int TRmax, int TCp, int NC, int NQL, bool smem_tile) {
     const int TRp = (TRmax + 31) & ~31;
+    const int RG = kWarps / NQL;
     size_t o = 0;
     auto take = [&](size_t bytes) {
       size_t r = o;
@@ -91,8 +109,8 @@ struct SeqSmem {
     ired = take(sizeof(int) * (kWarps + 1));
     cx = take(sizeof(double) * 4 * 4);
     misc = take(sizeof(double) * 32);
-    xd = take(sizeof(double) * 2 * NC);         // per-cluster fp64 records
-    xu = take(sizeof(uint32_t) * 6 * NC);       // per-cluster 32-bit records
+    xd = take(sizeof(double) * 2 * NC);    // per-cluster fp64 records
+    xu = take(sizeof(uint32_t) * 6 * NC);  // per-cluster 32-bit records
     tile = take(smem_tile ? sizeof(float) * (size_t)TRmax * TCp : 0);
     uval = take(sizeof(float) * TRp);
     ypart = take(sizeof(float) * 2 * TRp);
@@ -100,7 +118,7 @@ struct SeqSmem {
     rmax = take(sizeof(float) * TRp);
     rmaxv = take(sizeof(float) * TRp);
     rmaxj = take(sizeof(int) * TRp);
-    const size_t zb = sizeof(float) * (size_t)kWarps * TCp;
+    const size_t zb = sizeof(float) * (size_t)RG * TCp;
     const size_t yb = sizeof(float) * TRp;
     zred = take(zb > yb ? zb : yb);
     yfull = zred;
@@ -112,13 +130,13 @@ struct SeqSmem {
   }
 };
 
-// misc[] slots (doubles unless noted)
+// misc[] slots (doubles)
 enum {
   MS_E0 = 0,
   MS_R2,
   MS_M,      // entry score of the best single entry (as fp64)
   MS_MVAL,   // its signed value (fp32 held in fp64)
-  MS_MI,     // its row (int held in fp64)
+  MS_MI,     // its row
   MS_MJ,     // its column
   MS_ISTAR,  // starting row of the component
   MS_WIN,    // winning cluster
@@ -135,9 +153,9 @@ __device__ __forceinline__ float tern(float x, double thr) {
   return a > thr ? (x > 0.f ? 1.f : -1.f) : 0.f;
 }
 
-// Writes the packed bitplanes of the ternary values vals[0..len) (floats in
-// {-1,0,1}) covering global entries [g0, g0+len) with g0 % 32 == 0, into
-// plane0[g0/32 ..] and plane1 = plane0 + W.  One warp per word.
+// Packed bitplanes of the ternary values vals[0..len) (floats in {-1,0,1})
+// that stand for global entries [g0, g0+len), g0 % 32 == 0: plain stores into
+// plane0[g0/32 ..] and plane0[W + g0/32 ..].  One warp per word.
 __device__ __forceinline__ void pack_planes(const float* vals, int len, int g0, uint32_t* plane0,
                                             int W) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -154,6 +172,26 @@ __device__ __forceinline__ void pack_planes(const float* vals, int len, int g0, 
   }
 }
 
+// Same for an arbitrary start g0: words are shared with the neighbouring
+// bands, so the bits are OR-ed into zero-initialised planes.
+__device__ __forceinline__ void pack_planes_or(const float* vals, int len, int g0,
+                                               uint32_t* plane0, int W) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int w0 = g0 >> 5, w1 = (g0 + len + 31) >> 5;
+  for (int t = w0 + wid; t < w1; t += kWarps) {
+    const int e = t * 32 + lane - g0;
+    const float x = (e >= 0 && e < len) ? vals[e] : 0.f;
+    const uint32_t mk = __ballot_sync(0xffffffffu, x != 0.f);
+    const uint32_t sg = __ballot_sync(0xffffffffu, x < 0.f);
+    if (lane == 0) {
+      if (mk) atomicOr(plane0 + t, mk);
+      if (sg) atomicOr(plane0 + W + t, sg);
+    }
+  }
+}
+
+__device__ __forceinline__ long long tick() { return clock64(); }
+
 template <int NQL, bool SMT>
 __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
@@ -163,16 +201,17 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int m = a.m, n = a.n;
 
-  // ---- partition ----
-  const int ra = c * a.nchr / a.NC, rb = (c + 1) * a.nchr / a.NC;
-  const int r0 = ra * 32, r1 = min(rb * 32, m), TR = r1 - r0;
+  // ---- partition: rows split evenly over clusters, 32-column chunks over CTAs
+  const int r0 = (int)((long long)c * m / a.NC), r1 = (int)((long long)(c + 1) * m / a.NC);
+  const int TR = r1 - r0;
   const int ca = q * a.nchc / a.CS, cb = (q + 1) * a.nchc / a.CS;
   const int c0 = ca * 32, c1 = min(cb * 32, n), TC = c1 - c0;
   const int TCp = a.TCp;
   const int NQ = (TC + 3) >> 2;
   const int Wm = (m + 31) >> 5, Wn = (n + 31) >> 5;
+  constexpr int RG = kWarps / NQL;  // row groups of the z pass
 
-  const SeqSmem L(a.TRmax, TCp, a.NC, SMT);
+  const SeqSmem L(a.TRmax, TCp, a.NC, NQL, SMT);
   double* xd = (double*)(smem + L.xd);
   uint32_t* xu = (uint32_t*)(smem + L.xu);
   double* red = (double*)(smem + L.red);
@@ -196,12 +235,30 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
   const int TRp = (a.TRmax + 31) & ~31;
   const bool weighted = a.w != nullptr;
   const double tau = (double)a.tau;
+  const bool timer = blockIdx.x == 0 && tid == 0;
+  // phase accumulators live in shared memory (misc[16..]): one thread uses them
+  long long* ph = (long long*)(misc + 16);
+  if (timer) {
+    for (int p = 0; p < PH_N; ++p) ph[p] = 0;
+    ph[PH_N] = tick();
+  }
+  auto mark = [&](int p) {
+    if (timer) {
+      const long long t = tick();
+      ph[p] += t - ph[PH_N];
+      ph[PH_N] = t;
+    }
+  };
 
-  bool ab = false;  // this CTA gave up waiting
+  bool ab = false;  // this CTA gave up waiting (made block uniform at sync points)
   uint32_t ep = 0;  // exchange epoch (identical sequence in every CTA)
   auto slot = [&](uint32_t e) -> uint64_t* { return a.xbuf + (size_t)(e % 3u) * a.slot_words; };
   auto rec = [&](uint64_t* s, int cc, int qq) -> uint64_t* {
     return s + (size_t)(cc * a.CS + qq) * a.recw;
+  };
+  // payload of an already loaded word, or wait for it
+  auto take = [&](uint64_t v, const uint64_t* p) -> uint32_t {
+    return ((uint32_t)(v >> 32) == ep) ? (uint32_t)v : xw_wait(p, ep, ab, a.budget, a.abort_word);
   };
 
   // ---- setup: A -> tile, weights, validity ----
@@ -231,9 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
   }
   bad = block_sum_int(bad, ired) > 0 ? 1 : 0;
 
-  // Per-row statistics of this CTA's columns for rows with touched(i):
-  // rho_p[i] = sum_j w_j R_ij^2 (fp32), rmax/rmaxv/rmaxj = best entry score,
-  // its value and local column (lowest column on ties).
+  // Per-row statistics of this CTA's columns: rho_p[i] = sum_j w_j R_ij^2
+  // (fp32), rmax/rmaxv/rmaxj = best entry score, its value and its local
+  // column (lowest column on ties).  One warp per row.
   auto row_stats = [&](int i) {
     const float4* row = (const float4*)(T + (size_t)i * TCp);
     float rho = 0.f, bs = -1.f, bv = 0.f;
@@ -306,7 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       }
     }
     const double R2c = block_sum(r2, red);
-    // block argmax of (brho, bi) and of (bs, bflat)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const double orho = __shfl_xor_sync(0xffffffffu, brho, o);
@@ -371,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
         xw_store(mine + TCp + 10, ep, (uint32_t)bad_in);
       }
     }
-    // cluster records, one thread per cluster
+    // cluster records: one thread per cluster, its 9 words loaded together
     double* x_rho = xd;
     double* x_r2 = xd + a.NC;
     uint32_t* x_row = xu;
@@ -380,18 +436,20 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     float* x_bs = (float*)(xu + 3 * a.NC);
     float* x_bv = (float*)(xu + 4 * a.NC);
     for (int cc = tid; cc < a.NC; cc += kThreads) {
-      const uint64_t* r = rec(s, cc, 0) + TCp;
-      const uint32_t l2 = xw_wait(r + 2, ep, ab, a.budget, a.abort_word);
-      const uint32_t h2 = xw_wait(r + 3, ep, ab, a.budget, a.abort_word);
-      x_rho[cc] = u2d(l2, h2);
-      x_row[cc] = xw_wait(r + 4, ep, ab, a.budget, a.abort_word);
-      x_bs[cc] = u2f(xw_wait(r + 5, ep, ab, a.budget, a.abort_word));
-      x_flat[cc] = xw_wait(r + 6, ep, ab, a.budget, a.abort_word);
-      x_bv[cc] = u2f(xw_wait(r + 7, ep, ab, a.budget, a.abort_word));
-      const uint32_t l8 = xw_wait(r + 8, ep, ab, a.budget, a.abort_word);
-      const uint32_t h8 = xw_wait(r + 9, ep, ab, a.budget, a.abort_word);
-      x_r2[cc] = u2d(l8, h8);
-      x_bad[cc] = xw_wait(r + 10, ep, ab, a.budget, a.abort_word);
+      const uint64_t* r = rec(s, cc, 0) + TCp + 2;
+      uint64_t v[9];
+#pragma unroll
+      for (int b = 0; b < 9; ++b) v[b] = xw_load(r + b);
+      uint32_t p[9];
+#pragma unroll
+      for (int b = 0; b < 9; ++b) p[b] = take(v[b], r + b);
+      x_rho[cc] = u2d(p[0], p[1]);
+      x_row[cc] = p[2];
+      x_bs[cc] = u2f(p[3]);
+      x_flat[cc] = p[4];
+      x_bv[cc] = u2f(p[5]);
+      x_r2[cc] = u2d(p[6], p[7]);
+      x_bad[cc] = p[8];
     }
     ab = __syncthreads_or(ab);
     if (tid == 0) {
@@ -421,15 +479,15 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     int win = (int)misc[MS_WIN];
     win = (win >= 0 && win < a.NC) ? win : 0;
     // starting v for my columns: T_tau of the winning row
-    double rs = 0.0;
     if (tid < a.CS) {
       const uint64_t* r = rec(s, win, tid) + TCp;
-      const uint32_t lo = xw_wait(r, ep, ab, a.budget, a.abort_word);
-      const uint32_t hi = xw_wait(r + 1, ep, ab, a.budget, a.abort_word);
+      const uint64_t v0 = xw_load(r), v1 = xw_load(r + 1);
+      const uint32_t lo = take(v0, r), hi = take(v1, r + 1);
       red[tid] = u2d(lo, hi);
     }
     ab = __syncthreads_or(ab);
     if (tid == 0) {
+      double rs = 0.0;
       for (int qq = 0; qq < a.CS; ++qq) rs += red[qq];
       misc[MS_ROWSS] = rs;
     }
@@ -448,6 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
   if (tid == 0) misc[MS_E0] = misc[MS_R2];
   __syncthreads();
   const double E0 = misc[MS_E0];
+  mark(PH_SETUP);
 
   long long n_fb = 0, n_zero = 0;
   int tpos = 0;
@@ -457,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     // ---- cluster-uniform decision point ----
     if (tid == 0) misc[(comp & 1) ? MS_AB1 : MS_AB0] = ab ? 1.0 : 0.0;
     cl.sync();
-    int any_ab = 0;
     if (tid == 0) {
+      int any_ab = 0;
       for (int qq = 0; qq < a.CS; ++qq)
         any_ab |= cl.map_shared_rank(misc, qq)[(comp & 1) ? MS_AB1 : MS_AB0] != 0.0;
       misc[MS_ABORT] = (double)any_ab;
@@ -469,13 +528,9 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     if (comp > 0 && blockIdx.x == 0 && tid == 0)
       a.energy[comp - 1] = E0 > 0.0 ? 1.0 - misc[MS_R2] / E0 : 1.0;
     if (misc[MS_M] <= 0.0) {
-      // the residual vanished: the remaining components are empty
+      // the residual vanished: the remaining components are empty (packed_B
+      // was zeroed before the launch)
       for (int cc = comp; cc < a.k; ++cc) {
-        if (q == 0)
-          for (int t = (r0 >> 5) + tid; t < (r1 + 31) >> 5; t += kThreads) {
-            a.pB[(size_t)cc * 2 * Wm + t] = 0u;
-            a.pB[(size_t)cc * 2 * Wm + Wm + t] = 0u;
-          }
         for (int t = (c0 >> 5) + tid; t < (c1 + 31) >> 5; t += kThreads) {
           a.pC[(size_t)cc * 2 * Wn + t] = 0u;
           a.pC[(size_t)cc * 2 * Wn + Wn + t] = 0u;
@@ -494,6 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       pack_planes(vval, TC, c0, tb, Wn);
       if (blockIdx.x == 0 && tid == 0) a.trace_row[tpos] = (int32_t)misc[MS_ISTAR];
     }
+    mark(PH_STATS);
 
     int nu_total = 0;
     for (int it = 0; it < a.iters; ++it) {
@@ -550,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
           if (i0 + rr < TR) yp[i0 + rr] = v;
         }
       }
+      mark(PH_YPASS);
       cl.sync();
       // all-gather y over the cluster (fixed order), local sum of squares
       double ys = 0.0;
@@ -560,6 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
         ys += (double)s * (double)s;
       }
       const double Syc = block_sum(ys, red);
+      mark(PH_YGATHER);
       ++ep;
       {
         uint64_t* s = slot(ep);
@@ -569,8 +627,9 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
         }
         double* ysum = xd;
         for (int cc = tid; cc < a.NC; cc += kThreads) {
-          const uint32_t lo = xw_wait(rec(s, cc, 0) + 0, ep, ab, a.budget, a.abort_word);
-          const uint32_t hi = xw_wait(rec(s, cc, 0) + 1, ep, ab, a.budget, a.abort_word);
+          const uint64_t* r = rec(s, cc, 0);
+          const uint64_t v0 = xw_load(r), v1 = xw_load(r + 1);
+          const uint32_t lo = take(v0, r), hi = take(v1, r + 1);
           ysum[cc] = u2d(lo, hi);
         }
         ab = __syncthreads_or(ab);
@@ -588,59 +647,67 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
         uval[i] = uu;
         cnt += uu != 0.f;
       }
-      const int nnz_c = block_sum_int(cnt, ired);  // includes a __syncthreads
-      if (traced && q == 0) pack_planes(uval, TR, r0, tb + 2 * Wn + it * 2 * (Wm + Wn), Wm);
+      const int nnz_c = block_sum_int(cnt, ired);  // includes __syncthreads
+      if (traced && q == 0) pack_planes_or(uval, TR, r0, tb + 2 * Wn + it * 2 * (Wm + Wn), Wm);
+      mark(PH_YXCHG);
 
       // ---- z = R^T u over the cluster's rows, my columns ----
-      float4 za[NQL];
-#pragma unroll
-      for (int qi = 0; qi < NQL; ++qi) za[qi] = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int i = wid; i < TR; i += kWarps) {
-        const float ui = uval[i];
-        if (ui == 0.f) continue;
-        const float4* row = (const float4*)(T + (size_t)i * TCp);
-#pragma unroll
-        for (int qi = 0; qi < NQL; ++qi) {
-          const int quad = lane + 32 * qi;
+      // warp wid covers 128-column strip (wid % NQL) over row group (wid / NQL)
+      {
+        const int strip = wid % NQL, rgrp = wid / NQL;
+        const int quad = strip * 32 + lane;
+        if (rgrp < RG) {
+          float4 za = make_float4(0.f, 0.f, 0.f, 0.f);
           if (quad < NQ) {
-            const float4 r4 = row[quad];
-            za[qi].x = fmaf(ui, r4.x, za[qi].x);
-            za[qi].y = fmaf(ui, r4.y, za[qi].y);
-            za[qi].z = fmaf(ui, r4.z, za[qi].z);
-            za[qi].w = fmaf(ui, r4.w, za[qi].w);
+            for (int i = rgrp; i < TR; i += RG) {
+              const float ui = uval[i];
+              if (ui == 0.f) continue;
+              const float4 r4 = ((const float4*)(T + (size_t)i * TCp))[quad];
+              za.x = fmaf(ui, r4.x, za.x);
+              za.y = fmaf(ui, r4.y, za.y);
+              za.z = fmaf(ui, r4.z, za.z);
+              za.w = fmaf(ui, r4.w, za.w);
+            }
+            *(float4*)(zred + (size_t)rgrp * TCp + 4 * quad) = za;
           }
         }
       }
-#pragma unroll
-      for (int qi = 0; qi < NQL; ++qi) {
-        const int quad = lane + 32 * qi;
-        if (quad < NQ) *(float4*)(zred + (size_t)wid * TCp + 4 * quad) = za[qi];
-      }
       __syncthreads();
+      mark(PH_ZPASS);
       ++ep;
       {
         uint64_t* s = slot(ep);
         uint64_t* mine = rec(s, c, q);
         for (int j = tid; j < TC; j += kThreads) {
           float zs = 0.f;
-          for (int ww = 0; ww < kWarps; ++ww) zs += zred[(size_t)ww * TCp + j];
+          for (int g = 0; g < RG; ++g) zs += zred[(size_t)g * TCp + j];
           xw_store(mine + j, ep, f2u(zs));
         }
         if (tid == 0) xw_store(mine + TCp, ep, (uint32_t)nnz_c);
         double zz = 0.0;
         for (int j = tid; j < TC; j += kThreads) {
           float z = 0.f;
-          for (int cc = 0; cc < a.NC; ++cc)
-            z += u2f(xw_wait(rec(s, cc, q) + j, ep, ab, a.budget, a.abort_word));
+          for (int cc0 = 0; cc0 < a.NC; cc0 += 8) {
+            uint64_t v[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+              if (cc0 + b < a.NC) v[b] = xw_load(rec(s, cc0 + b, q) + j);
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+              if (cc0 + b < a.NC) z += u2f(take(v[b], rec(s, cc0 + b, q) + j));
+          }
           zfull[j] = z;
           zz += (double)z * (double)z;
         }
-        for (int cc = tid; cc < a.NC; cc += kThreads)
-          nnzu[cc] = (int)xw_wait(rec(s, cc, q) + TCp, ep, ab, a.budget, a.abort_word);
+        for (int cc = tid; cc < a.NC; cc += kThreads) {
+          const uint64_t* r = rec(s, cc, q) + TCp;
+          nnzu[cc] = (int)take(xw_load(r), r);
+        }
         ab = __syncthreads_or(ab);
         const double Szq = block_sum(zz, red);
         if (tid == 0) cx[buf * 4 + 0] = Szq;
       }
+      mark(PH_ZXCHG);
       cl.sync();
       double Sz = 0.0;
       for (int qq = 0; qq < a.CS; ++qq) Sz += cl.map_shared_rank(cx, qq)[buf * 4 + 0];
@@ -654,6 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       __syncthreads();
       nu_total = ired[kWarps];
       if (traced) pack_planes(vval, TC, c0, tb + 2 * Wn + it * 2 * (Wm + Wn) + 2 * Wm, Wn);
+      mark(PH_ZSYNC);
     }
 
     // ---- scale, gain, safeguard ----
@@ -697,9 +765,10 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     if (traced) ++tpos;
 
     // ---- emit ----
-    if (q == 0) pack_planes(uval, TR, r0, a.pB + (size_t)comp * 2 * Wm, Wm);
+    if (q == 0) pack_planes_or(uval, TR, r0, a.pB + (size_t)comp * 2 * Wm, Wm);
     pack_planes(vval, TC, c0, a.pC + (size_t)comp * 2 * Wn, Wn);
     if (blockIdx.x == 0 && tid == 0) a.D[comp] = d;
+    mark(PH_SCALE);
 
     // ---- deflate R <- R - d u v^T, refresh touched rows' statistics ----
     for (int i = wid; i < TR; i += kWarps) {
@@ -724,7 +793,9 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       row_stats(i);
     }
     __syncthreads();
+    mark(PH_DEFLATE);
     stats_exchange(0);
+    mark(PH_STATS);
   }
 
   // final energy entry, counters, status
@@ -737,6 +808,9 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       a.stats[1] = n_zero;
       a.stats[2] = a.NC;
       a.stats[3] = a.CS;
+      a.stats[4] = SMT ? 1 : 0;
+      a.stats[5] = (long long)gridDim.x;
+      for (int p = 0; p < PH_N; ++p) a.stats[kStatPhase0 + p] = ph[p];
     }
     if (misc[MS_BAD] != 0.0) atomicCAS(a.dev_status, 0, EXTERND_ERR_NONFINITE);
   }
@@ -753,8 +827,8 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
 // ---------------------------------------------------------------------------
 
 template <int NQL, bool SMT>
-static cudaError_t launch_one(const SeqArgs& args, size_t smem, cudaStream_t st, int* max_clusters_out,
-                              bool query_only) {
+static cudaError_t launch_one(const SeqArgs& args, size_t smem, cudaStream_t st,
+                              int* max_clusters_out, bool query_only) {
   auto kern = seq_als_kernel<NQL, SMT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -836,6 +910,10 @@ struct SeqPlan {
   size_t smem = 0;
 };
 
+// Chooses cluster size, cluster count and tile residency.  Candidates must be
+// co-resident (occupancy query).  Shared-memory residency of the whole
+// residual wins; among equals the estimated cost per half-step, tile words
+// streamed per CTA plus the cross-cluster words each CTA polls, is smallest.
 static cudaError_t plan_seq(int m, int n, cudaStream_t st, SeqPlan* out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -843,14 +921,14 @@ static cudaError_t plan_seq(int m, int n, cudaStream_t st, SeqPlan* out) {
   int nsm = 0, optin = 0;
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  const int nchr = (m + 31) / 32, nchc = (n + 31) / 32;
+  const int nchc = (n + 31) / 32;
   int force_cs = 0;
   if (const char* s = getenv("EXTERND_CLUSTER")) force_cs = atoi(s);
-  const int cands[5] = {16, 8, 4, 2, 1};
+  const int cands[] = {16, 12, 10, 9, 8, 6, 5, 4, 3, 2, 1};
   SeqPlan best;
-  double best_score = -1.0;
-  for (int ci = 0; ci < 5; ++ci) {
-    int CS = cands[ci];
+  double best_cost = 1e300;
+  bool best_smt = false;
+  for (int CS : cands) {
     if (force_cs > 0 && CS != force_cs) continue;
     if (CS > nchc) continue;
     const int colchunks = (nchc + CS - 1) / CS;
@@ -858,13 +936,13 @@ static cudaError_t plan_seq(int m, int n, cudaStream_t st, SeqPlan* out) {
     const int TCp = (TC + 3) & ~3;
     const int NQL = nql_for(TCp);
     if (NQL > 8) continue;
-    int NC = std::min(std::min(nchr, 64), std::max(1, nsm / CS));
     for (int smt_try = 1; smt_try >= 0; --smt_try) {
       const bool smt = smt_try == 1;
-      int nc = NC;
-      for (int guard = 0; guard < 8 && nc >= 1; ++guard) {
-        const int TRmax = std::min(((nchr + nc - 1) / nc) * 32, m);
-        SeqSmem L(TRmax, TCp, nc, smt);
+      if (best_smt && !smt) continue;
+      int nc = std::min(std::min(m, 64), std::max(1, nsm / CS));
+      for (int guard = 0; guard < 16 && nc >= 1; ++guard) {
+        const int TRmax = (m + nc - 1) / nc;
+        SeqSmem L(TRmax, TCp, nc, NQL, smt);
         const size_t stat = static_smem(NQL, smt);
         if (L.total + stat > (size_t)optin) break;
         SeqArgs probe = {};
@@ -878,10 +956,11 @@ static cudaError_t plan_seq(int m, int n, cudaStream_t st, SeqPlan* out) {
           break;
         }
         if (maxc >= nc) {
-          // prefer shared-memory residency, then more SMs, then larger clusters
-          const double score = (smt ? 1e6 : 0.0) + (double)(nc * CS) + 0.01 * CS;
-          if (score > best_score) {
-            best_score = score;
+          const double tile_w = (double)TRmax * TCp * (smt ? 1.0 : 4.0);
+          const double cost = tile_w + 8.0 * nc * TCp;
+          if ((smt && !best_smt) || cost < best_cost) {
+            best_cost = cost;
+            best_smt = smt;
             best.NC = nc;
             best.CS = CS;
             best.TRmax = TRmax;
@@ -900,6 +979,46 @@ static cudaError_t plan_seq(int m, int n, cudaStream_t st, SeqPlan* out) {
   if (best.NC == 0) return cudaErrorNotSupported;
   *out = best;
   return cudaSuccess;
+}
+
+static void fill_args(SeqArgs& a, const SeqHostArgs& h, const SeqPlan& pl, int recw,
+                      long long slot_words) {
+  a.A = h.A;
+  a.m = (int)h.m;
+  a.n = (int)h.n;
+  a.k = (int)h.k;
+  a.tau = h.tau;
+  a.iters = h.iters;
+  a.w = h.w;
+  a.pB = h.packed_B;
+  a.pC = h.packed_C;
+  a.D = h.D;
+  a.energy = h.energy;
+  a.NC = pl.NC;
+  a.CS = pl.CS;
+  a.nchc = (a.n + 31) / 32;
+  a.TRmax = pl.TRmax;
+  a.TCp = pl.TCp;
+  a.recw = recw;
+  a.slot_words = slot_words;
+  a.trace_comp = h.trace_comp;
+  a.ntrace = (int)h.ntrace;
+  a.trace_bits = h.trace_bits;
+  a.trace_row = h.trace_row;
+  a.trace_flags = h.trace_flags;
+  a.stats = h.stats;
+  a.budget = h.wait_budget > 0 ? h.wait_budget : kDefaultWaitBudget;
+}
+
+// Zero-initialises what the kernel ORs into.
+static cudaError_t clear_outputs(const SeqHostArgs& h, cudaStream_t st) {
+  const size_t Wm = (size_t)((h.m + 31) / 32), Wn = (size_t)((h.n + 31) / 32);
+  cudaError_t e = cudaMemsetAsync(h.packed_B, 0, sizeof(uint32_t) * 2 * Wm * (size_t)h.k, st);
+  if (e == cudaSuccess && h.ntrace > 0 && h.trace_bits)
+    e = cudaMemsetAsync(h.trace_bits, 0,
+                        sizeof(uint32_t) * (size_t)h.ntrace * (2 * Wn + (size_t)h.iters * 2 * (Wm + Wn)),
+                        st);
+  return e;
 }
 
 int seq_decompose(const SeqHostArgs& h, cudaStream_t st) {
@@ -922,36 +1041,12 @@ int seq_decompose(const SeqHostArgs& h, cudaStream_t st) {
   }
   int rc = EXTERND_OK;
   if (cudaMemsetAsync(ws, 0, tile_off, st) != cudaSuccess) rc = EXTERND_ERR_CUDA;
+  if (rc == EXTERND_OK && clear_outputs(h, st) != cudaSuccess) rc = EXTERND_ERR_CUDA;
   if (rc == EXTERND_OK) {
     SeqArgs a = {};
-    a.A = h.A;
-    a.m = (int)h.m;
-    a.n = (int)h.n;
-    a.k = (int)h.k;
-    a.tau = h.tau;
-    a.iters = h.iters;
-    a.w = h.w;
-    a.pB = h.packed_B;
-    a.pC = h.packed_C;
-    a.D = h.D;
-    a.energy = h.energy;
-    a.NC = pl.NC;
-    a.CS = pl.CS;
-    a.nchr = (a.m + 31) / 32;
-    a.nchc = (a.n + 31) / 32;
-    a.TRmax = pl.TRmax;
-    a.TCp = pl.TCp;
-    a.recw = recw;
+    fill_args(a, h, pl, recw, slot_words);
     a.gtile = pl.smt ? nullptr : (float*)((char*)ws + tile_off);
     a.xbuf = (uint64_t*)ws;
-    a.slot_words = slot_words;
-    a.trace_comp = h.trace_comp;
-    a.ntrace = (int)h.ntrace;
-    a.trace_bits = h.trace_bits;
-    a.trace_row = h.trace_row;
-    a.trace_flags = h.trace_flags;
-    a.stats = h.stats;
-    a.budget = h.wait_budget > 0 ? h.wait_budget : kDefaultWaitBudget;
     a.abort_word = (int*)((char*)ws + abort_off);
     a.dev_status = status_word_ptr();
     if (!a.dev_status) rc = EXTERND_ERR_CUDA;
@@ -968,7 +1063,6 @@ int seq_decompose(const SeqHostArgs& h, cudaStream_t st) {
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == EXTERND_OK) rc = EXTERND_ERR_CUDA;
   return rc;
 }
-
 
 // Same launch as seq_decompose, but the exchange ring and the abort word live
 // in caller-provided device scratch instead of a cudaMallocAsync workspace,
@@ -988,31 +1082,11 @@ int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scrat
   const size_t need = abort_off + 256;
   if (need > scratch_bytes) return EXTERND_ERR_SCRATCH_LIMIT;
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return EXTERND_ERR_CUDA;
+  if (clear_outputs(h, st) != cudaSuccess) return EXTERND_ERR_CUDA;
   SeqArgs a = {};
-  a.A = h.A;
-  a.m = (int)h.m;
-  a.n = (int)h.n;
-  a.k = (int)h.k;
-  a.tau = h.tau;
-  a.iters = h.iters;
-  a.w = h.w;
-  a.pB = h.packed_B;
-  a.pC = h.packed_C;
-  a.D = h.D;
-  a.energy = h.energy;
-  a.NC = pl.NC;
-  a.CS = pl.CS;
-  a.nchr = (a.m + 31) / 32;
-  a.nchc = (a.n + 31) / 32;
-  a.TRmax = pl.TRmax;
-  a.TCp = pl.TCp;
-  a.recw = recw;
+  fill_args(a, h, pl, recw, slot_words);
   a.gtile = nullptr;
   a.xbuf = (uint64_t*)scratch;
-  a.slot_words = slot_words;
-  a.trace_comp = nullptr;
-  a.ntrace = 0;
-  a.budget = kDefaultWaitBudget;
   a.abort_word = (int*)((char*)scratch + abort_off);
   a.dev_status = status_word_ptr();
   if (!a.dev_status) return EXTERND_ERR_CUDA;

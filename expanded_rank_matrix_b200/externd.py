@@ -161,7 +161,7 @@ class Trace:
     bits: torch.Tensor  # [ntrace, S] int32
     row: torch.Tensor   # [ntrace] int32
     flags: torch.Tensor  # [ntrace] uint8
-    stats: torch.Tensor  # [4] int64
+    stats: torch.Tensor  # [16] int64 (see externd_decompose_traced)
     iters: int
 
 
@@ -180,7 +180,7 @@ def decompose_traced(A: torch.Tensor, mu: float, tau: float, iters: int,
     tb = torch.zeros((max(nt, 1), S), dtype=torch.int32, device=dev)
     tr = torch.zeros(max(nt, 1), dtype=torch.int32, device=dev)
     tf = torch.zeros(max(nt, 1), dtype=torch.uint8, device=dev)
-    stats = torch.zeros(4, dtype=torch.int64, device=dev)
+    stats = torch.zeros(16, dtype=torch.int64, device=dev)
     rc = load().externd_decompose_traced(
         _ptr(A), m, n, mu, tau, iters, _ptr(w), 1, _ptr(out.packed_B), _ptr(out.packed_C),
         _ptr(out.D), _ptr(out.energy), nt, _ptr(tc), _ptr(tb) if nt else None,

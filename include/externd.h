@@ -107,9 +107,13 @@ int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau,
  *   trace_row    [ntrace] int32 out: the starting row i*.
  *   trace_flags  [ntrace] uint8 out: bit 0 = the safeguard replaced the ALS
  *                pair of this component.
- *   stats        [4] int64 out or NULL: [0] safeguard activations over all
+ *   stats        [16] int64 out or NULL: [0] safeguard activations over all
  *                components, [1] components emitted as zero because the
- *                residual vanished, [2] launch clusters, [3] CTAs per cluster.
+ *                residual vanished, [2] launch clusters, [3] CTAs per cluster,
+ *                [4] 1 if the residual stayed in shared memory, [5] CTAs,
+ *                [6..15] SM cycles CTA 0 spent per phase (setup, R W v pass,
+ *                cluster gather of y, y exchange, R^T u pass, z exchange,
+ *                z cluster step, scale and emit, deflation, statistics).
  *   wait_budget  upper bound, in SM clock cycles, on every device-side wait
  *                for another CTA's data; 0 selects the default (about 1 s).
  *                A wait that runs out sets EXTERND_ERR_TIMEOUT and the kernel
