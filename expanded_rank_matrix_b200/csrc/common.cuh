@@ -61,6 +61,49 @@ __device__ __forceinline__ uint32_t xw_wait(const uint64_t* p, uint32_t epoch, b
   }
 }
 
+// Waits for `count` (<= N) words base[t * stride], t < count, all tagged with
+// `epoch`, and writes their payloads to out[].  All words are loaded back to
+// back; every later round re-loads all words still stale together, so each
+// round costs one memory round trip however many words it covers.  Bounded
+// like xw_wait.
+template <int N>
+__device__ __forceinline__ void xw_wait_n(const uint64_t* base, long long stride, int count,
+                                          uint32_t epoch, uint32_t (&out)[N], bool& ab,
+                                          long long budget, int* abort_word) {
+  uint64_t v[N];
+  unsigned pending = 0u;
+#pragma unroll
+  for (int t = 0; t < N; ++t)
+    if (t < count) v[t] = xw_load(base + t * stride);
+#pragma unroll
+  for (int t = 0; t < N; ++t)
+    if (t < count && (uint32_t)(v[t] >> 32) != epoch) pending |= 1u << t;
+  if (pending && !ab) {
+    const long long t0 = clock64();
+    unsigned spins = 0;
+    while (pending) {
+#pragma unroll
+      for (int t = 0; t < N; ++t)
+        if ((pending >> t) & 1u) v[t] = xw_load(base + t * stride);
+#pragma unroll
+      for (int t = 0; t < N; ++t)
+        if (((pending >> t) & 1u) && (uint32_t)(v[t] >> 32) == epoch) pending &= ~(1u << t);
+      if (!pending) break;
+      if (((++spins) & 63u) == 0u && ld_flag(abort_word) != 0) {
+        ab = true;
+        break;
+      }
+      if (clock64() - t0 > budget) {
+        atomicCAS(abort_word, 0, EXTERND_ERR_TIMEOUT);
+        ab = true;
+        break;
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < N; ++t) out[t] = (t < count && !ab) ? (uint32_t)v[t] : 0u;
+}
+
 __device__ __forceinline__ uint32_t f2u(float x) { return __float_as_uint(x); }
 __device__ __forceinline__ float u2f(uint32_t x) { return __uint_as_float(x); }
 __device__ __forceinline__ uint32_t dlo(double x) { return (uint32_t)__double_as_longlong(x); }

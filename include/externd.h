@@ -110,7 +110,8 @@ int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau,
  *   stats        [16] int64 out or NULL: [0] safeguard activations over all
  *                components, [1] components emitted as zero because the
  *                residual vanished, [2] launch clusters, [3] CTAs per cluster,
- *                [4] 1 if the residual stayed in shared memory, [5] CTAs,
+ *                [4] rows of each CTA's residual tile kept in shared memory,
+ *                [5] rows of each CTA's tile (the rest stream from global memory),
  *                [6..15] SM cycles CTA 0 spent per phase (setup, R W v pass,
  *                cluster gather of y, y exchange, R^T u pass, z exchange,
  *                z cluster step, scale and emit, deflation, statistics).
