@@ -44,7 +44,7 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
   if (k < 1) return EXTERND_ERR_INVALID_ARG;
   if (!(tau >= 0.0f) || !std::isfinite(tau)) return EXTERND_ERR_INVALID_ARG;
   if (iters < 1 || iters > 1000) return EXTERND_ERR_INVALID_ARG;
-  if (block < 1 || block > 256 || block > k || block > (m < n ? m : n)) return EXTERND_ERR_INVALID_ARG;
+  if (block < 1 || block > 64 || block > k || block > (m < n ? m : n)) return EXTERND_ERR_INVALID_ARG;
   if (ntrace < 0 || wait_budget < 0) return EXTERND_ERR_INVALID_ARG;
   if (ntrace > 0 && (!trace_comp || !trace_bits || !trace_row || !trace_flags || block != 1))
     return EXTERND_ERR_INVALID_ARG;
@@ -63,6 +63,31 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
   b.A = A; b.m = m; b.n = n; b.k = k; b.tau = tau; b.iters = iters; b.w = w; b.block = block;
   b.packed_B = packed_B; b.packed_C = packed_C; b.D = D; b.energy = energy_trace; b.stats = stats;
   return externd::block_decompose(b, st);
+}
+
+int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float mu, float tau,
+                                   int iters, const float* w, int block, uint32_t* packed_B,
+                                   uint32_t* packed_C, float* D, double* energy_trace,
+                                   int64_t ntrace, const int64_t* trace_block, uint64_t* trace_uv,
+                                   int32_t* trace_rows, externd_stream_t stream) {
+  if (block < 2) return EXTERND_ERR_INVALID_ARG;
+  if (ntrace < 0 || (ntrace > 0 && (!trace_block || !trace_uv || !trace_rows)))
+    return EXTERND_ERR_INVALID_ARG;
+  if (!A || !packed_B || !packed_C || !D || !energy_trace) return EXTERND_ERR_INVALID_ARG;
+  if (!aligned4(A) || !aligned4(packed_B) || !aligned4(packed_C) || !aligned4(D) ||
+      ((uintptr_t)energy_trace & 7u) || (w && !aligned4(w)) || ((uintptr_t)trace_uv & 7u))
+    return EXTERND_ERR_INVALID_ARG;
+  if (!sizes_ok(m, n)) return EXTERND_ERR_INVALID_ARG;
+  const int64_t k = externd_rank(m, n, mu);
+  if (k < 1) return EXTERND_ERR_INVALID_ARG;
+  if (!(tau >= 0.0f) || !std::isfinite(tau)) return EXTERND_ERR_INVALID_ARG;
+  if (iters < 1 || iters > 1000) return EXTERND_ERR_INVALID_ARG;
+  if (block > 64 || block > k || block > (m < n ? m : n)) return EXTERND_ERR_INVALID_ARG;
+  externd::BlockHostArgs b = {};
+  b.A = A; b.m = m; b.n = n; b.k = k; b.tau = tau; b.iters = iters; b.w = w; b.block = block;
+  b.packed_B = packed_B; b.packed_C = packed_C; b.D = D; b.energy = energy_trace;
+  b.ntrace = ntrace; b.trace_block = trace_block; b.trace_uv = trace_uv; b.trace_rows = trace_rows;
+  return externd::block_decompose(b, (cudaStream_t)stream);
 }
 
 int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,

@@ -37,6 +37,10 @@ struct BlockHostArgs {
   float* D;
   double* energy;
   int64_t* stats;
+  int64_t ntrace;
+  const int64_t* trace_block;  // host array: traced block indices
+  uint64_t* trace_uv;          // device: per traced block, V0 then U_t, V_t masks
+  int32_t* trace_rows;         // device: per traced block, the start rows
 };
 
 int seq_decompose(const SeqHostArgs& h, cudaStream_t st);
@@ -44,6 +48,12 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st);
 int reconstruct(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
                 int64_t k, float* out, cudaStream_t st);
 int* status_word_ptr();
+int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
+                   const unsigned long long* Vs, const float* w, int bb, int klen, int splits,
+                   float* Pp, cudaStream_t st);
+int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
+                    const unsigned long long* Us, int bb, int klen, int splits, float* Qp,
+                    cudaStream_t st);
 int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
                                cudaStream_t st);
 

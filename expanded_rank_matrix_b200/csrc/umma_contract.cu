@@ -1,0 +1,413 @@
+// Block-ALS contractions on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+//   P  = R (W V)   : M = rows of R,    N = 64 components, K = columns of R
+//   Q^T = R^T U    : M = columns of R, N = 64 components, K = rows of R
+//
+// The ternary operand (V or U, entries -1/0/+1) is exact in bf16.  The fp32
+// residual (times w_j for P when weighted, one fp32 rounding) is split exactly
+// into three bf16 parts hi + mid + lo (8 + 8 + 8 significand bits), so every
+// product the tensor core forms is exact and only its fp32 accumulation rounds
+// -- the same class of error as an fp32 dot product on the CUDA cores.
+//
+// Per CTA: one 128 x 64 fp32 accumulator in tensor memory; the K range of the
+// CTA's split is walked in chunks of 32, double buffered in shared memory:
+// all threads convert a chunk into the canonical no-swizzle UMMA layouts while
+// the tensor core runs the 3 x 2 MMAs (3 parts x K/16 steps) of the previous
+// chunk, issued by one thread; tcgen05.commit on a per-stage mbarrier tells when a stage may be
+// refilled.  Every mbarrier wait is bounded; a wait that runs out records
+// EXTERND_ERR_TIMEOUT, the CTA stops issuing, drains (bounded) and frees its
+// tensor memory.  Outputs are split-K partials Xp[split][row][64].
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace externd {
+namespace umma {
+
+typedef unsigned long long u64;
+
+constexpr int kM = 128;      // accumulator rows (TMEM lanes)
+constexpr int kN = 64;       // components (TMEM columns)
+constexpr int kKc = 32;      // K chunk
+constexpr int kThreads = 256;
+constexpr int kPartBytes = kM * kKc * 2;   // one bf16 part of the A chunk: 8 KB
+constexpr int kBBytes = kN * kKc * 2;      // B chunk: 4 KB
+constexpr int kSboK = 8 * kKc * 2;         // K-major: bytes between 8-row groups
+constexpr int kLboMN = kM / 8 * 128;       // MN-major: bytes between 8-k groups
+constexpr int kStageBytes = 3 * kPartBytes + kBBytes;
+constexpr int kSmemBytes = 2 * kStageBytes + 1024;  // 56 KB + alignment slack: 3-4 CTAs per SM
+constexpr long long kWaitBudget = 2000000000LL;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// --- tcgen05 / mbarrier wrappers (PTX ISA, sm_100a) ---
+__device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(addr), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0u;
+}
+// bounded wait for completion of the phase with the given parity
+__device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity) {
+  if (mbar_test(addr, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_test(addr, parity))
+    if (clock64() - t0 > kWaitBudget) return false;
+  return true;
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t mbar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, no swizzle: start address, leading-dimension
+// byte offset (LBO), stride-dimension byte offset (SBO), version 1.
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3fffu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  return d;                // base offset 0, legacy LBO mode, layout type 0 (no swizzle)
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, M x N.
+__host__ __device__ constexpr uint32_t make_idesc(int a_mn_major) {
+  return (1u << 4)                      // D format: f32
+         | (1u << 7)                    // A format: bf16
+         | (1u << 10)                   // B format: bf16
+         | ((uint32_t)a_mn_major << 15)  // A major: 0 = K, 1 = MN
+         | (0u << 16)                   // B major: K
+         | ((uint32_t)(kN >> 3) << 17)  // N / 8
+         | ((uint32_t)(kM >> 4) << 24);  // M / 16
+}
+
+// exact three-way bf16 split of an fp32 value
+__device__ __forceinline__ void split3(float x, __nv_bfloat16& h, __nv_bfloat16& md,
+                                       __nv_bfloat16& l) {
+  h = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(h);
+  md = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(md);
+  l = __float2bfloat16_rn(r2);
+}
+
+__device__ __forceinline__ uint32_t pack2(__nv_bfloat16 a, __nv_bfloat16 b) {
+  return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+}
+
+// K-major no-swizzle offset of element (row, k) of a [rows x kKc] bf16 tile:
+// core matrices of 8 rows x 16 B; K-adjacent cores 128 B apart (LBO),
+// 8-row groups kSboK bytes apart (SBO).
+__device__ __forceinline__ uint32_t kmaj_off(int row, int k) {
+  return (uint32_t)((row >> 3) * kSboK + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+// MN-major no-swizzle offset of element (mn, k) of a [128 x kKc] bf16 tile:
+// core matrices of 8 k-rows x 16 B (8 mn); MN-adjacent cores 128 B apart (SBO),
+// K groups of 8 kLboMN bytes apart (LBO).
+__device__ __forceinline__ uint32_t mnmaj_off(int mn, int k) {
+  return (uint32_t)((mn >> 3) * 128 + (k >> 3) * kLboMN + (k & 7) * 16 + (mn & 7) * 2);
+}
+
+// Ternary B chunk: element (l, k) = sign of component l at K index k0+k, from
+// 64-bit masks; K-major layout, 16 bytes (8 k) per store.
+__device__ __forceinline__ void fill_b(unsigned char* bs, const u64* __restrict__ Mk,
+                                       const u64* __restrict__ Sg, int k0, int klim) {
+  constexpr int kGroups = kKc / 8;  // 8-element K groups per chunk
+  for (int e = threadIdx.x; e < kN * kGroups; e += kThreads) {
+    const int l = e / kGroups, kg = e - l * kGroups;
+    uint32_t w[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      uint32_t v = 0u;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int k = kg * 8 + 2 * h + t;
+        uint32_t bits = 0u;
+        if (k0 + k < klim) {
+          const u64 mk = Mk[k0 + k];
+          if ((mk >> l) & 1ull) bits = ((Sg[k0 + k] >> l) & 1ull) ? 0xBF80u : 0x3F80u;
+        }
+        v |= bits << (16 * t);
+      }
+      w[h] = v;
+    }
+    *(uint4*)(bs + kmaj_off(l, kg * 8)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// MODE 0: P = R (W V) -- A = R rows [i0, i0+128), K = columns; K-major A.
+// MODE 1: Q^T = R^T U -- A = R^T columns [i0, i0+128), K = rows; MN-major A.
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1) contract_kernel(
+    const float* __restrict__ R, int m, int n, const u64* __restrict__ Mk,
+    const u64* __restrict__ Sg, const float* __restrict__ w, int bb, int klen,
+    float* __restrict__ Xp, int* __restrict__ status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // 1024-byte aligned base for the operand tiles
+  unsigned char* smem = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ uint32_t tmem_base;
+  __shared__ __align__(8) u64 mbar[2];
+  __shared__ int bad;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int M = MODE == 0 ? m : n;  // output rows
+  const int Kdim = MODE == 0 ? n : m;
+  const int i0 = blockIdx.x * kM;
+  const int split = blockIdx.y;
+  const int k_begin = split * klen, k_end = min(Kdim, k_begin + klen);
+  const int nchunks = k_end > k_begin ? (k_end - k_begin + kKc - 1) / kKc : 0;
+  // 16-byte loads only when every row of R starts 16-byte aligned
+  const bool vec4 = (n & 3) == 0 && (((uintptr_t)R) & 15) == 0;
+
+  if (wid == 0) {
+    tmem_alloc(smem_u32(&tmem_base), kN);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(smem_u32(&mbar[0]), 1);
+    mbar_init(smem_u32(&mbar[1]), 1);
+    fence_mbar_init();
+    bad = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const uint32_t idesc = make_idesc(MODE);
+  bool ok = true;
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int s = c & 1;
+    unsigned char* stage = smem + s * kStageBytes;
+    if (c >= 2) {  // the MMAs that read this stage (chunk c-2) must be done
+      if (tid == 0 && !mbar_wait(smem_u32(&mbar[s]), (uint32_t)((c / 2 - 1) & 1))) bad = 1;
+      __syncthreads();
+      if (bad) {
+        ok = false;
+        break;
+      }
+    }
+    const int k0 = k_begin + c * kKc;
+    // ---- A chunk: fp32 -> hi/mid/lo bf16, canonical layout ----
+    if (MODE == 0) {
+      // tile rows r (128) x k (kKc = 32): lanes cover 8 rows x 16 k per step
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = (wid + 8 * (u & 1)) * 8 + (lane >> 2);
+        const int k = (u >> 1) * 16 + (lane & 3) * 4;
+        const int gi = i0 + r, gk = k0 + k;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (gi < m) {
+          const float* src = R + (size_t)gi * n + gk;
+          if (vec4 && gk + 3 < k_end) {
+            const float4 v = *(const float4*)src;
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (gk + e < k_end) x[e] = src[e];
+          }
+          if (w) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (gk + e < k_end) x[e] *= w[gk + e];
+          }
+        }
+        __nv_bfloat16 h[4], md[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split3(x[e], h[e], md[e], lo[e]);
+        const uint32_t off = kmaj_off(r, k);
+        *(uint2*)(stage + off) = make_uint2(pack2(h[0], h[1]), pack2(h[2], h[3]));
+        *(uint2*)(stage + kPartBytes + off) = make_uint2(pack2(md[0], md[1]), pack2(md[2], md[3]));
+        *(uint2*)(stage + 2 * kPartBytes + off) =
+            make_uint2(pack2(lo[0], lo[1]), pack2(lo[2], lo[3]));
+      }
+    } else {
+      // tile mn = columns j (128) x k = rows i (kKc = 32): lanes cover 8 k x 16 mn per step
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int k = (lane >> 2) + 8 * u;
+        const int mn = wid * 16 + (lane & 3) * 4;
+        const int gi = k0 + k, gj = i0 + mn;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (gi < k_end) {
+          const float* src = R + (size_t)gi * n + gj;
+          if (vec4 && gj + 3 < n) {
+            const float4 v = *(const float4*)src;
+            x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (gj + e < n) x[e] = src[e];
+          }
+        }
+        __nv_bfloat16 h[4], md[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split3(x[e], h[e], md[e], lo[e]);
+        const uint32_t off = mnmaj_off(mn, k);
+        *(uint2*)(stage + off) = make_uint2(pack2(h[0], h[1]), pack2(h[2], h[3]));
+        *(uint2*)(stage + kPartBytes + off) = make_uint2(pack2(md[0], md[1]), pack2(md[2], md[3]));
+        *(uint2*)(stage + 2 * kPartBytes + off) =
+            make_uint2(pack2(lo[0], lo[1]), pack2(lo[2], lo[3]));
+      }
+    }
+    // ---- B chunk: ternary components ----
+    fill_b(stage + 3 * kPartBytes, Mk, Sg, k0, k_end);
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t abase = smem_u32(stage), bbase = smem_u32(stage + 3 * kPartBytes);
+#pragma unroll
+      for (int p = 0; p < 3; ++p)
+#pragma unroll
+        for (int ks = 0; ks < kKc / 16; ++ks) {
+          uint64_t ad, bd;
+          if (MODE == 0)
+            ad = make_desc(abase + p * kPartBytes + ks * 256, 128, kSboK);
+          else
+            ad = make_desc(abase + p * kPartBytes + ks * 2 * kLboMN, kLboMN, 128);
+          bd = make_desc(bbase + ks * 256, 128, kSboK);
+          umma_bf16(tmem, ad, bd, idesc, (c > 0 || p > 0 || ks > 0) ? 1u : 0u);
+        }
+      umma_commit(smem_u32(&mbar[s]));
+    }
+  }
+  // ---- wait for the last chunk's MMAs (all earlier ones complete before) ----
+  if (tid == 0 && nchunks > 0) {
+    const int cl = ok ? nchunks - 1 : -1;
+    if (cl >= 0) {
+      if (!mbar_wait(smem_u32(&mbar[cl & 1]), (uint32_t)((cl / 2) & 1))) bad = 1;
+    } else {
+      // stopped early: drain whatever was issued (bounded)
+      for (int s = 0; s < 2; ++s) mbar_wait(smem_u32(&mbar[s]), 0u);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (bad) {
+    if (tid == 0) atomicCAS(status, 0, EXTERND_ERR_TIMEOUT);
+  } else if (nchunks > 0) {
+    // ---- epilogue: TMEM -> partials; warp w reads lanes 32*(w%4).., columns 32*(w/4).. ----
+    const int q = wid & 3, chalf = wid >> 2;
+    const int row = q * 32 + lane;
+    const int gi = i0 + row;
+    float* out = Xp + ((size_t)split * M + gi) * bb;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t v[16];
+      const int col = chalf * 32 + h * 16;
+      tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col, v);
+      if (gi < M)
+#pragma unroll
+        for (int t = 0; t < 16; ++t)
+          if (col + t < bb) out[col + t] = __uint_as_float(v[t]);
+    }
+  } else {
+    // empty K range: zero partials
+    const int q = wid & 3, chalf = wid >> 2;
+    const int gi = i0 + q * 32 + lane;
+    if (gi < M)
+      for (int t = 0; t < 32; ++t)
+        if (chalf * 32 + t < bb) Xp[((size_t)split * M + gi) * bb + chalf * 32 + t] = 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (wid == 0) tmem_dealloc(tmem, kN);
+}
+
+}  // namespace umma
+
+// Host launchers; klen must be a multiple of kKc (32).
+int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
+                   const unsigned long long* Vs, const float* w, int bb, int klen, int splits,
+                   float* Pp, cudaStream_t st) {
+  using namespace umma;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(contract_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaFuncSetAttribute(contract_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    attr = true;
+  }
+  int* status = status_word_ptr();
+  dim3 grid((unsigned)((m + kM - 1) / kM), (unsigned)splits);
+  contract_kernel<0><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Vm, Vs, w, bb, klen, Pp, status);
+  return cudaGetLastError() == cudaSuccess ? EXTERND_OK : EXTERND_ERR_CUDA;
+}
+
+int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
+                    const unsigned long long* Us, int bb, int klen, int splits, float* Qp,
+                    cudaStream_t st) {
+  using namespace umma;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(contract_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaFuncSetAttribute(contract_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    attr = true;
+  }
+  int* status = status_word_ptr();
+  dim3 grid((unsigned)((n + kM - 1) / kM), (unsigned)splits);
+  contract_kernel<1><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Um, Us, nullptr, bb, klen, Qp,
+                                                        status);
+  return cudaGetLastError() == cudaSuccess ? EXTERND_OK : EXTERND_ERR_CUDA;
+}
+
+}  // namespace externd

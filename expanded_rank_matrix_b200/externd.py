@@ -28,7 +28,8 @@ ERR_SCRATCH_LIMIT = -7
 
 # every symbol include/externd.h declares
 EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_traced",
-           "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc")
+           "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc",
+           "externd_decompose_block_traced")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -63,6 +64,10 @@ def load(path: str = LIB_PATH):
     L.externd_decompose_noalloc.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
                                             ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp]
     L.externd_decompose_noalloc.restype = ctypes.c_int
+    L.externd_decompose_block_traced.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
+                                                 ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp,
+                                                 _vp, _i64, _vp, _vp, _vp, _vp]
+    L.externd_decompose_block_traced.restype = ctypes.c_int
     L.externd_sync_status.argtypes = [_vp]
     L.externd_sync_status.restype = ctypes.c_int
     _lib = L
@@ -238,3 +243,61 @@ def trace_vectors(tr: Trace, t_idx: int, m: int, n: int):
         vs.append(unpack_planes(b[off:off + 2 * Wn].reshape(2, Wn), n))
         off += 2 * Wn
     return v0, us, vs
+
+
+@dataclass
+class BlockTrace:
+    blocks: np.ndarray     # traced block indices
+    uv: torch.Tensor       # [ntrace, 2n + iters*2(m+n)] int64 masks
+    rows: torch.Tensor     # [ntrace, block] int32
+    iters: int
+    block: int
+
+
+def decompose_block_traced(A: torch.Tensor, mu: float, tau: float, iters: int, block: int,
+                           trace_blocks: Sequence[int], w: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None, check: bool = True):
+    m, n = A.shape
+    k = rank(m, n, mu)
+    out = alloc_factors(m, n, k, A.device)
+    nblocks = (k + block - 1) // block
+    blocks = np.array(sorted(set(int(b) for b in trace_blocks if 0 <= b < nblocks)), np.int64)
+    nt = int(blocks.size)
+    words_ = 2 * n + iters * 2 * (m + n)
+    uv = torch.zeros((max(nt, 1), words_), dtype=torch.int64, device=A.device)
+    rows = torch.zeros((max(nt, 1), block), dtype=torch.int32, device=A.device)
+    rc = load().externd_decompose_block_traced(
+        _ptr(A), m, n, mu, tau, iters, _ptr(w), block, _ptr(out.packed_B), _ptr(out.packed_C),
+        _ptr(out.D), _ptr(out.energy), nt,
+        blocks.ctypes.data_as(ctypes.c_void_p) if nt else None, _ptr(uv) if nt else None,
+        _ptr(rows) if nt else None, _stream(stream))
+    if rc != OK:
+        raise ExterndError(rc, "externd_decompose_block_traced")
+    status = sync_status(stream)
+    if check and status != OK:
+        raise ExterndError(status, "externd_decompose_block_traced (device)")
+    return out, BlockTrace(blocks, uv[:nt], rows[:nt], iters, block)
+
+
+def _mask_codes(mask: np.ndarray, sign: np.ndarray, bb: int) -> np.ndarray:
+    """[len] uint64 masks -> [bb, len] int8 codes."""
+    mk = mask.view(np.uint64)[None, :] >> np.arange(bb, dtype=np.uint64)[:, None]
+    sg = sign.view(np.uint64)[None, :] >> np.arange(bb, dtype=np.uint64)[:, None]
+    mk = (mk & np.uint64(1)).astype(np.int8)
+    sg = (sg & np.uint64(1)).astype(np.int8)
+    return (mk * (1 - 2 * sg)).astype(np.int8)
+
+
+def block_trace_vectors(tr: BlockTrace, t_idx: int, m: int, n: int, bb: int):
+    """Traced block t_idx -> (rows[bb], V0 [bb, n], [U_t [bb, m]], [V_t [bb, n]])."""
+    a = tr.uv[t_idx].cpu().numpy()
+    rows = tr.rows[t_idx].cpu().numpy()[:bb].astype(np.int64)
+    V0 = _mask_codes(a[:n], a[n:2 * n], bb)
+    us, vs = [], []
+    off = 2 * n
+    for _ in range(tr.iters):
+        us.append(_mask_codes(a[off:off + m], a[off + m:off + 2 * m], bb))
+        off += 2 * m
+        vs.append(_mask_codes(a[off:off + n], a[off + n:off + 2 * n], bb))
+        off += 2 * n
+    return rows, V0, us, vs

@@ -79,7 +79,7 @@ int64_t externd_rank(int64_t m, int64_t n, float mu);
  *   iters        ALS iterations per component (or per block), >= 1.
  *   w            [n] fp32 per-input-column importance weights, finite and
  *                > 0, or NULL for the unweighted objective.
- *   block        1 (sequential) or 2..min(k, 256) (block-ALS).
+ *   block        1 (sequential) or 2..min(k, m, n, 64) (block-ALS).
  *   packed_B     [k][2][ceil(m/32)] uint32 out.
  *   packed_C     [k][2][ceil(n/32)] uint32 out.
  *   D            [k] fp32 out.
@@ -126,6 +126,28 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
                              const int64_t* trace_comp, uint32_t* trace_bits, int32_t* trace_row,
                              uint8_t* trace_flags, int64_t* stats, int64_t wait_budget,
                              externd_stream_t stream);
+
+/*
+ * externd_decompose_block_traced -- externd_decompose with block >= 2 plus a
+ * record of the block-ALS trajectory of selected blocks (used to compare the
+ * device path with a reference half-step by half-step).  Block t covers
+ * components t*block .. min(k, (t+1)*block) - 1; bit l of a mask word stands
+ * for the block's component l.
+ *
+ *   trace_block  [ntrace] int64 HOST array of block indices (may be NULL when
+ *                ntrace == 0).
+ *   trace_uv     [ntrace][2n + iters*2(m+n)] uint64 (device) out: per traced
+ *                block the n mask words then the n sign words of the starting
+ *                V, then for t = 1..iters the m mask and m sign words of U_t
+ *                and the n mask and n sign words of V_t.
+ *   trace_rows   [ntrace][block] int32 (device) out: the block's start rows in
+ *                order (energy descending, index ascending).
+ */
+int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float mu, float tau,
+                                   int iters, const float* w, int block, uint32_t* packed_B,
+                                   uint32_t* packed_C, float* D, double* energy_trace,
+                                   int64_t ntrace, const int64_t* trace_block, uint64_t* trace_uv,
+                                   int32_t* trace_rows, externd_stream_t stream);
 
 /*
  * externd_reconstruct -- A_hat = B diag(D) C from the packed factors (the

@@ -326,11 +326,128 @@ void orc_top_rows(const double* rho, int64_t m, int64_t b, int64_t* rows) {
   for (int64_t l = 0; l < b; ++l) rows[l] = idx[l];
 }
 
+// Block-ALS U half-step (paper Sec. 2.4 per [PITH]; the U-step target is the
+// reading R W V (V^T W V + eps I)^-1): U = T_col of that target, each column
+// thresholded with its own rms over the m rows.  V and U are column-major
+// per component: V[l*n + j], U[l*m + i].  targets (m x bb, row-major, may be
+// NULL) receives the target, thr (bb, may be NULL) the thresholds.
+void orc_block_u_step(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* V,
+                      const float* w, double tau, int8_t* U, double* targets, double* thr) {
+  std::vector<double> G(bb * bb);
+  for (int64_t l = 0; l < bb; ++l)
+    for (int64_t l2 = 0; l2 < bb; ++l2) {
+      double s = 0.0;
+      for (int64_t j = 0; j < n; ++j) s += wt(w, j) * V[l * n + j] * V[l2 * n + j];
+      G[l * bb + l2] = s;
+    }
+  const double eps = ridge_eps(G, bb);
+  for (int64_t l = 0; l < bb; ++l) G[l * bb + l] += eps;
+  // P = R W V (m x bb); targets are the rows of P solved against G: G t_i = p_i
+  std::vector<double> Pt(bb * m);
+  for (int64_t i = 0; i < m; ++i)
+    for (int64_t l = 0; l < bb; ++l) {
+      double s = 0.0;
+      for (int64_t j = 0; j < n; ++j)
+        if (V[l * n + j]) s += (double)R[i * n + j] * wt(w, j) * V[l * n + j];
+      Pt[l * m + i] = s;
+    }
+  chol_solve(G, bb, Pt, m);
+  for (int64_t l = 0; l < bb; ++l) {
+    const double t = orc_ternarize(&Pt[l * m], m, tau, U + l * m);
+    if (thr) thr[l] = t;
+    if (targets)
+      for (int64_t i = 0; i < m; ++i) targets[i * bb + l] = Pt[l * m + i];
+  }
+}
+
+// Block-ALS V half-step (Eq. 3): V = T_col(((U^T U + eps I)^-1 U^T R)^T).
+void orc_block_v_step(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* U,
+                      double tau, int8_t* V, double* targets, double* thr) {
+  std::vector<double> G(bb * bb);
+  for (int64_t l = 0; l < bb; ++l)
+    for (int64_t l2 = 0; l2 < bb; ++l2) {
+      double s = 0.0;
+      for (int64_t i = 0; i < m; ++i) s += (double)(U[l * m + i] * U[l2 * m + i]);
+      G[l * bb + l2] = s;
+    }
+  const double eps = ridge_eps(G, bb);
+  for (int64_t l = 0; l < bb; ++l) G[l * bb + l] += eps;
+  std::vector<double> Q(bb * n, 0.0);  // U^T R
+  for (int64_t l = 0; l < bb; ++l)
+    for (int64_t i = 0; i < m; ++i) {
+      const int8_t ui = U[l * m + i];
+      if (!ui) continue;
+      for (int64_t j = 0; j < n; ++j) Q[l * n + j] += (double)ui * (double)R[i * n + j];
+    }
+  chol_solve(G, bb, Q, n);
+  for (int64_t l = 0; l < bb; ++l) {
+    const double t = orc_ternarize(&Q[l * n], n, tau, V + l * n);
+    if (thr) thr[l] = t;
+    if (targets)
+      for (int64_t j = 0; j < n; ++j) targets[j * bb + l] = Q[l * n + j];
+  }
+}
+
+// Joint block scales: (G + eps I) D = r with G = (U^T U) o (V^T W V) and
+// r_l = u_l^T R W v_l, over the components whose u and v are both nonzero
+// (the others take d = 0).  Also returns G (raw, bb x bb) and r.
+void orc_block_scales(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* U,
+                      const int8_t* V, const float* w, double* D, double* Graw, double* r) {
+  std::vector<double> GU(bb * bb), GV(bb * bb), G(bb * bb);
+  for (int64_t l = 0; l < bb; ++l)
+    for (int64_t l2 = 0; l2 < bb; ++l2) {
+      double su = 0.0, sv = 0.0;
+      for (int64_t i = 0; i < m; ++i) su += (double)(U[l * m + i] * U[l2 * m + i]);
+      for (int64_t j = 0; j < n; ++j) sv += wt(w, j) * V[l * n + j] * V[l2 * n + j];
+      GU[l * bb + l2] = su;
+      GV[l * bb + l2] = sv;
+    }
+  for (int64_t l = 0; l < bb; ++l) {
+    double s = 0.0;
+    for (int64_t i = 0; i < m; ++i) {
+      const int8_t ui = U[l * m + i];
+      if (!ui) continue;
+      for (int64_t j = 0; j < n; ++j)
+        if (V[l * n + j]) s += (double)ui * (double)R[i * n + j] * wt(w, j) * V[l * n + j];
+    }
+    r[l] = s;
+  }
+  for (int64_t l = 0; l < bb * bb; ++l) G[l] = GU[l] * GV[l];
+  for (int64_t l = 0; l < bb * bb; ++l) Graw[l] = G[l];
+  const double eps = ridge_eps(G, bb);
+  std::vector<int64_t> act;
+  for (int64_t l = 0; l < bb; ++l)
+    if (GU[l * bb + l] > 0.0 && GV[l * bb + l] > 0.0) act.push_back(l);
+  for (int64_t l = 0; l < bb; ++l) D[l] = 0.0;
+  if (!act.empty()) {
+    const int64_t na = (int64_t)act.size();
+    std::vector<double> Ga(na * na), ra(na);
+    for (int64_t a = 0; a < na; ++a) {
+      ra[a] = r[act[a]];
+      for (int64_t c = 0; c < na; ++c) Ga[a * na + c] = G[act[a] * bb + act[c]];
+      Ga[a * na + a] += eps;
+    }
+    chol_solve(Ga, na, ra, 1);
+    for (int64_t a = 0; a < na; ++a) D[act[a]] = ra[a];
+  }
+}
+
+// Starting V of a block: column l = T_tau(R[rows[l], :]) (each row's own rms).
+void orc_block_init(const float* R, int64_t m, int64_t n, int64_t bb, const int64_t* rows,
+                    double tau, int8_t* V) {
+  std::vector<double> row(n);
+  for (int64_t l = 0; l < bb; ++l) {
+    for (int64_t j = 0; j < n; ++j) row[j] = (double)R[rows[l] * n + j];
+    orc_ternarize(row.data(), n, tau, V + l * n);
+  }
+}
+
 // Block-ALS with decorrelated least-squares targets (paper Sec. 2.4, Eq. 3 per
 // [PITH]; [REV] "Method": batched block-ALS).  Fits bb = min(b, k - c0)
-// components per sweep.  Outputs as orc_decompose_seq; energy per component
-// from the closed form |R|^2 - 2 sum d_l r_l + sum d_l d_l' G_ll' over the
-// block prefix.
+// components per sweep: start from the bb largest-energy rows, `iters`
+// rounds of the U and V half-steps above, joint scales, then bb ordered
+// rank-1 deflations.  Energy per component from the closed form
+// |R|^2 - 2 sum d_l r_l + sum d_l d_l' G_ll' over the block prefix.
 void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
                          const float* w, int64_t b, int8_t* U, int8_t* V, float* D,
                          double* energy, int64_t* init_row) {
@@ -342,117 +459,23 @@ void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double
     orc_row_norms(R.data(), m, n, w, rho.data());
     std::vector<int64_t> rows(bb);
     orc_top_rows(rho.data(), m, bb, rows.data());
-    std::vector<int8_t> Ub(m * bb, 0), Vb(n * bb, 0);  // column l of U is Ub[i*bb+l]
-    std::vector<double> col(std::max(m, n));
-    std::vector<int8_t> code(std::max(m, n));
-    for (int64_t l = 0; l < bb; ++l) {
-      init_row[c0 + l] = rows[l];
-      for (int64_t j = 0; j < n; ++j) col[j] = (double)R[rows[l] * n + j];
-      orc_ternarize(col.data(), n, tau, code.data());
-      for (int64_t j = 0; j < n; ++j) Vb[j * bb + l] = code[j];
-    }
-    std::vector<double> G(bb * bb), P, Q;
+    for (int64_t l = 0; l < bb; ++l) init_row[c0 + l] = rows[l];
+    std::vector<int8_t> Ub(bb * m, 0), Vb(bb * n, 0);
+    orc_block_init(R.data(), m, n, bb, rows.data(), tau, Vb.data());
     for (int t = 0; t < iters; ++t) {
-      // U-step: P = R W V, target P (V^T W V + eps I)^-1, threshold per column.
-      for (int64_t l = 0; l < bb; ++l)
-        for (int64_t l2 = 0; l2 < bb; ++l2) {
-          double s = 0.0;
-          for (int64_t j = 0; j < n; ++j) s += wt(w, j) * Vb[j * bb + l] * Vb[j * bb + l2];
-          G[l * bb + l2] = s;
-        }
-      double eps = ridge_eps(G, bb);
-      for (int64_t l = 0; l < bb; ++l) G[l * bb + l] += eps;
-      P.assign(m * bb, 0.0);
-      for (int64_t i = 0; i < m; ++i)
-        for (int64_t l = 0; l < bb; ++l) {
-          double s = 0.0;
-          for (int64_t j = 0; j < n; ++j)
-            if (Vb[j * bb + l]) s += (double)R[i * n + j] * wt(w, j) * Vb[j * bb + l];
-          P[i * bb + l] = s;
-        }
-      // rows of P^T solved against the symmetric system: T = P G^-1 <=> G T^T = P^T
-      std::vector<double> Pt(bb * m);
-      for (int64_t i = 0; i < m; ++i)
-        for (int64_t l = 0; l < bb; ++l) Pt[l * m + i] = P[i * bb + l];
-      std::vector<double> Gc = G;
-      chol_solve(Gc, bb, Pt, m);
-      for (int64_t l = 0; l < bb; ++l) {
-        orc_ternarize(&Pt[l * m], m, tau, code.data());
-        for (int64_t i = 0; i < m; ++i) Ub[i * bb + l] = code[i];
-      }
-      // V-step (Eq. 3): V = T_col(((U^T U + eps I)^-1 U^T R)^T).
-      for (int64_t l = 0; l < bb; ++l)
-        for (int64_t l2 = 0; l2 < bb; ++l2) {
-          double s = 0.0;
-          for (int64_t i = 0; i < m; ++i) s += (double)(Ub[i * bb + l] * Ub[i * bb + l2]);
-          G[l * bb + l2] = s;
-        }
-      eps = ridge_eps(G, bb);
-      for (int64_t l = 0; l < bb; ++l) G[l * bb + l] += eps;
-      Q.assign(bb * n, 0.0);
-      for (int64_t l = 0; l < bb; ++l)
-        for (int64_t i = 0; i < m; ++i) {
-          int8_t ui = Ub[i * bb + l];
-          if (!ui) continue;
-          for (int64_t j = 0; j < n; ++j) Q[l * n + j] += (double)ui * (double)R[i * n + j];
-        }
-      Gc = G;
-      chol_solve(Gc, bb, Q, n);
-      for (int64_t l = 0; l < bb; ++l) {
-        orc_ternarize(&Q[l * n], n, tau, code.data());
-        for (int64_t j = 0; j < n; ++j) Vb[j * bb + l] = code[j];
-      }
+      orc_block_u_step(R.data(), m, n, bb, Vb.data(), w, tau, Ub.data(), nullptr, nullptr);
+      orc_block_v_step(R.data(), m, n, bb, Ub.data(), tau, Vb.data(), nullptr, nullptr);
     }
-    // Joint scales: (G + eps I) D = r with G = (U^T U) o (V^T W V).
-    std::vector<double> GU(bb * bb), GV(bb * bb), r(bb, 0.0);
-    for (int64_t l = 0; l < bb; ++l)
-      for (int64_t l2 = 0; l2 < bb; ++l2) {
-        double su = 0.0, sv = 0.0;
-        for (int64_t i = 0; i < m; ++i) su += (double)(Ub[i * bb + l] * Ub[i * bb + l2]);
-        for (int64_t j = 0; j < n; ++j) sv += wt(w, j) * Vb[j * bb + l] * Vb[j * bb + l2];
-        GU[l * bb + l2] = su;
-        GV[l * bb + l2] = sv;
-      }
-    for (int64_t l = 0; l < bb; ++l) {
-      double s = 0.0;
-      for (int64_t i = 0; i < m; ++i) {
-        int8_t ui = Ub[i * bb + l];
-        if (!ui) continue;
-        for (int64_t j = 0; j < n; ++j)
-          if (Vb[j * bb + l]) s += (double)ui * (double)R[i * n + j] * wt(w, j) * Vb[j * bb + l];
-      }
-      r[l] = s;
-    }
-    for (int64_t l = 0; l < bb; ++l)
-      for (int64_t l2 = 0; l2 < bb; ++l2) G[l * bb + l2] = GU[l * bb + l2] * GV[l * bb + l2];
-    std::vector<double> Graw = G;
-    double eps = ridge_eps(G, bb);
-    // components with an empty u or v take d = 0 and drop out of the system
-    std::vector<int64_t> act;
-    for (int64_t l = 0; l < bb; ++l)
-      if (GU[l * bb + l] > 0.0 && GV[l * bb + l] > 0.0) act.push_back(l);
-    std::vector<double> dsol(bb, 0.0);
-    if (!act.empty()) {
-      int64_t na = (int64_t)act.size();
-      std::vector<double> Ga(na * na), ra(na);
-      for (int64_t a = 0; a < na; ++a) {
-        ra[a] = r[act[a]];
-        for (int64_t c = 0; c < na; ++c) Ga[a * na + c] = G[act[a] * bb + act[c]];
-        Ga[a * na + a] += eps;
-      }
-      chol_solve(Ga, na, ra, 1);
-      for (int64_t a = 0; a < na; ++a) dsol[act[a]] = ra[a];
-    }
+    std::vector<double> dsol(bb), Graw(bb * bb), r(bb);
+    orc_block_scales(R.data(), m, n, bb, Ub.data(), Vb.data(), w, dsol.data(), Graw.data(),
+                     r.data());
     std::vector<float> dl(bb);
     for (int64_t l = 0; l < bb; ++l) dl[l] = (float)dsol[l];
-    double base = orc_sumsq(R.data(), m, n, w);
-    std::vector<int8_t> uc(m), vc(n);
+    const double base = orc_sumsq(R.data(), m, n, w);
     for (int64_t l = 0; l < bb; ++l) {
-      for (int64_t i = 0; i < m; ++i) uc[i] = Ub[i * bb + l];
-      for (int64_t j = 0; j < n; ++j) vc[j] = Vb[j * bb + l];
-      orc_deflate(R.data(), m, n, uc.data(), vc.data(), dl[l]);
-      std::memcpy(U + (c0 + l) * m, uc.data(), m);
-      std::memcpy(V + (c0 + l) * n, vc.data(), n);
+      orc_deflate(R.data(), m, n, &Ub[l * m], &Vb[l * n], dl[l]);
+      std::memcpy(U + (c0 + l) * m, &Ub[l * m], m);
+      std::memcpy(V + (c0 + l) * n, &Vb[l * n], n);
       D[c0 + l] = dl[l];
       double e = base;
       for (int64_t a = 0; a <= l; ++a) {

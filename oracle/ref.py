@@ -56,6 +56,14 @@ def lib():
         L.orc_reconstruct.restype = None
         L.orc_top_rows.argtypes = [_D, _i64, _i64, _I64]
         L.orc_top_rows.restype = None
+        L.orc_block_u_step.argtypes = [_F, _i64, _i64, _i64, _I8, _F, ctypes.c_double, _I8, _D, _D]
+        L.orc_block_u_step.restype = None
+        L.orc_block_v_step.argtypes = [_F, _i64, _i64, _i64, _I8, ctypes.c_double, _I8, _D, _D]
+        L.orc_block_v_step.restype = None
+        L.orc_block_scales.argtypes = [_F, _i64, _i64, _i64, _I8, _I8, _F, _D, _D, _D]
+        L.orc_block_scales.restype = None
+        L.orc_block_init.argtypes = [_F, _i64, _i64, _i64, _I64, ctypes.c_double, _I8]
+        L.orc_block_init.restype = None
         L.orc_decompose_block.argtypes = [_F, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _F,
                                           _i64, _I8, _I8, _F, _D, _I64]
         L.orc_decompose_block.restype = None
@@ -210,3 +218,48 @@ def top_rows(rho, b: int):
     rows = np.empty(b, np.int64)
     lib().orc_top_rows(_p(rho, _D), rho.shape[0], b, _p(rows, _I64))
     return rows
+
+
+# --- block-ALS half-steps (component-major codes: U[l, i], V[l, j]) ---------
+
+def block_init(R, rows, tau):
+    R = _f32(R)
+    m, n = R.shape
+    rows = np.ascontiguousarray(rows, np.int64)
+    V = np.zeros((rows.shape[0], n), np.int8)
+    lib().orc_block_init(_p(R, _F), m, n, rows.shape[0], _p(rows, _I64), tau, _p(V, _I8))
+    return V
+
+
+def block_u_step(R, V, tau, w=None):
+    R = _f32(R); w = _f32(w)
+    m, n = R.shape
+    V = np.ascontiguousarray(V, np.int8)
+    bb = V.shape[0]
+    U = np.zeros((bb, m), np.int8)
+    T = np.zeros((m, bb)); thr = np.zeros(bb)
+    lib().orc_block_u_step(_p(R, _F), m, n, bb, _p(V, _I8), _p(w, _F), tau, _p(U, _I8), _p(T, _D),
+                           _p(thr, _D))
+    return U, T, thr
+
+
+def block_v_step(R, U, tau):
+    R = _f32(R)
+    m, n = R.shape
+    U = np.ascontiguousarray(U, np.int8)
+    bb = U.shape[0]
+    V = np.zeros((bb, n), np.int8)
+    T = np.zeros((n, bb)); thr = np.zeros(bb)
+    lib().orc_block_v_step(_p(R, _F), m, n, bb, _p(U, _I8), tau, _p(V, _I8), _p(T, _D), _p(thr, _D))
+    return V, T, thr
+
+
+def block_scales(R, U, V, w=None):
+    R = _f32(R); w = _f32(w)
+    m, n = R.shape
+    U = np.ascontiguousarray(U, np.int8); V = np.ascontiguousarray(V, np.int8)
+    bb = U.shape[0]
+    D = np.zeros(bb); G = np.zeros((bb, bb)); r = np.zeros(bb)
+    lib().orc_block_scales(_p(R, _F), m, n, bb, _p(U, _I8), _p(V, _I8), _p(w, _F), _p(D, _D),
+                           _p(G, _D), _p(r, _D))
+    return D, G, r

@@ -22,6 +22,10 @@ def _workloads():
         "llm1024_tau0.5": lambda: W.config_llm1024(0.5),
         "llm1024_tau0.7": lambda: W.config_llm1024(0.7),
         "attn2560": W.config_attn2560,
+        "mlp9728_b64": lambda: W.config_mlp9728(64),
+        "mlp9728_b1": lambda: W.config_mlp9728(1),
+        **{f"blk_{nm}": (lambda i=i: W.config_block_matrices(64)[i])
+           for i, (nm, _, _) in enumerate(W.BLOCK_MATRICES)},
     }
 
 
@@ -49,7 +53,7 @@ if __name__ == "__main__":
     data = json.load(open(OUT)) if os.path.exists(OUT) else {}
     data["_source"] = ("CPU oracle (oracle/externd_ref.cpp), free-running, single thread; "
                        "written by tests/golden/make_oracle_energy.py")
-    with ProcessPoolExecutor(max_workers=min(len(names), 5)) as ex:
+    with ProcessPoolExecutor(max_workers=min(len(names), 7)) as ex:
         for name, rec in ex.map(run, names):
             data[name] = rec
             print(name, rec["final_energy"], f"{rec['oracle_seconds']:.1f}s", flush=True)

@@ -109,3 +109,61 @@ def check_component(oracle, rep: Report, c: int, R: np.ndarray, E0: float, tau: 
     if abs(res_g - res_o) > NORM_RTOL * res_o + 1e-12 * E0:
         rep.fail(f"comp {c}: residual |R|^2 {res_g} vs oracle {res_o}")
     return Rn
+
+
+D_RTOL_BLOCK = 1e-5  # joint block scales (same bound as the sequential scales)
+
+
+@dataclass
+class BlockReport(Report):
+    blocks: int = 0
+    d_rel_max: float = 0.0
+
+
+def check_block(oracle, rep: "BlockReport", c0: int, R: np.ndarray, E0: float, tau: float,
+                iters: int, w, rows, V0, us, vs, U_emit, V_emit, D_gpu, E_gpu) -> np.ndarray:
+    """Teacher-forced check of one block (components c0 .. c0+bb-1) given R = R_c0;
+    returns the residual after replaying the device's block."""
+    bb = len(D_gpu)
+    rep.blocks += 1
+    rep.comps += bb
+    rho, _ = oracle.row_norms(R, w)
+    top = oracle.top_rows(rho, bb)
+    if not np.array_equal(np.sort(rows), np.sort(top)):
+        # allowed only where energies tie to rounding
+        if not np.allclose(np.sort(rho[rows])[::-1], rho[top], rtol=1e-12, atol=0):
+            rep.fail(f"block {c0}: start rows are not the {bb} largest-energy rows")
+        rep.init_ties += 1
+    if np.any(np.diff(rho[rows]) > 1e-12 * rho[rows][:-1]):
+        rep.fail(f"block {c0}: start rows not in descending energy order")
+    V0o = oracle.block_init(R, rows, tau)
+    for l in range(bb):
+        x = R[rows[l]].astype(np.float64)
+        thr = tau * np.sqrt(np.mean(x * x))
+        _cmp(rep, f"block {c0} v0[{l}]", V0[l], V0o[l], x, thr)
+    Vprev = V0
+    for t in range(iters):
+        Uo, T, thr = oracle.block_u_step(R, Vprev, tau, w)
+        for l in range(bb):
+            _cmp(rep, f"block {c0} u{t + 1}[{l}]", us[t][l], Uo[l], T[:, l], thr[l])
+        Vo, T, thr = oracle.block_v_step(R, us[t], tau)
+        for l in range(bb):
+            _cmp(rep, f"block {c0} v{t + 1}[{l}]", vs[t][l], Vo[l], T[:, l], thr[l])
+        Vprev = vs[t]
+    if not (np.array_equal(U_emit, us[-1]) and np.array_equal(V_emit, vs[-1])):
+        rep.fail(f"block {c0}: emitted factors differ from the last iterates")
+    Do, G, r = oracle.block_scales(R, us[-1], vs[-1], w)
+    for l in range(bb):
+        err = abs(float(D_gpu[l]) - Do[l])
+        if Do[l] != 0.0:
+            rep.d_rel_max = max(rep.d_rel_max, err / abs(Do[l]))
+        if err > D_RTOL_BLOCK * abs(Do[l]) + 1e-30:
+            rep.fail(f"block {c0}: scale {l} {D_gpu[l]} vs oracle {Do[l]}")
+    Rn = R
+    for l in range(bb):
+        Rn = oracle.deflate(Rn, U_emit[l], V_emit[l], D_gpu[l])
+    res_o = oracle.sumsq(Rn, w)
+    res_g = (1.0 - float(E_gpu[-1])) * E0
+    if abs(res_g - res_o) > NORM_RTOL * res_o + 1e-12 * E0:
+        rep.fail(f"block {c0}: residual |R|^2 {res_g} vs replay {res_o}")
+    return Rn

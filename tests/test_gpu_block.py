@@ -1,0 +1,108 @@
+"""Parity of the CUDA block-ALS path (block >= 2) with the CPU oracle through
+the C ABI: every traced block is checked half-step by half-step from the
+device's own iterates (teacher forced).  Needs a B200."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from expanded_rank_matrix_b200 import externd as X
+from expanded_rank_matrix_b200 import workloads as W
+from tests.parity import BlockReport, check_block
+
+pytestmark = pytest.mark.gpu
+
+FREE_ENERGY_ATOL = 1e-4
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def block_teacher_forced(oracle, A, mu, tau, iters, b, blocks=None, w=None):
+    m, n = A.shape
+    k = X.rank(m, n, mu)
+    nb = (k + b - 1) // b
+    blocks = list(range(nb)) if blocks is None else sorted(set(blocks))
+    f, tr = X.decompose_block_traced(_dev(A), mu, tau, iters, b, blocks,
+                                     w=None if w is None else _dev(w))
+    U, V, D, E = X.to_codes(f)
+    E0 = oracle.sumsq(A, w)
+    rep = BlockReport()
+    R = np.array(A, dtype=np.float32, copy=True)
+    at = 0
+    for ti, blk in enumerate(tr.blocks.tolist()):
+        c0 = blk * b
+        bb = min(b, k - c0)
+        oracle.replay_range(R, U, V, D, at, c0)
+        rows, V0, us, vs = X.block_trace_vectors(tr, ti, m, n, bb)
+        R = check_block(oracle, rep, c0, R, E0, tau, iters, w, rows, V0, us, vs,
+                        U[c0:c0 + bb], V[c0:c0 + bb], D[c0:c0 + bb], E[c0:c0 + bb])
+        at = c0 + bb
+    return rep, f
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_small_every_block(oracle, weighted):
+    A = W.llm_like(192, 160, 91, n_outliers=4)
+    w = W.lognormal_weights(160, 91) if weighted else None
+    rep, f = block_teacher_forced(oracle, A, 2.0, 0.5, 3, 16, w=w)
+    print(f"192x160 b=16 weighted={weighted}: {rep.blocks} blocks, band {rep.band_total} "
+          f"(mismatch {rep.band_mismatch}), max D rel err {rep.d_rel_max:.2e}")
+    assert rep.ok, rep.bad
+    ref = oracle.decompose(A, f.k, 0.5, 3, w=w, block=16)
+    assert abs(float(f.energy[-1]) - ref.energy[-1]) <= FREE_ENERGY_ATOL
+
+
+def test_ragged_last_block_and_max_block(oracle):
+    A = W.iid_gaussian(100, 90, 5)
+    rep, f = block_teacher_forced(oracle, A, 1.0, 0.5, 2, 16)   # k = 90: last block 10
+    assert rep.ok, rep.bad
+    A2 = W.llm_like(130, 128, 6, n_outliers=2)
+    rep2, f2 = block_teacher_forced(oracle, A2, 1.0, 0.5, 2, 64, blocks=[0, 1])
+    assert rep2.ok, rep2.bad
+
+
+def test_llm1024_sampled_blocks_and_free_running(oracle):
+    wl = W.config_llm1024(0.5)
+    rep, f = block_teacher_forced(oracle, wl.a, wl.mu, wl.tau, wl.iters, 64,
+                                  blocks=[0, 1, 12, 23])
+    print(f"llm1024 b=64: band {rep.band_total} mismatch {rep.band_mismatch} "
+          f"max D rel {rep.d_rel_max:.2e} ties {rep.init_ties}")
+    assert rep.ok, rep.bad
+    ref = oracle.decompose(wl.a, wl.k, wl.tau, wl.iters, block=64)
+    E = f.energy.cpu().numpy()
+    print(f"  final energy device {E[-1]:.8f} oracle {ref.energy[-1]:.8f}")
+    assert abs(E[-1] - ref.energy[-1]) <= FREE_ENERGY_ATOL
+
+
+def test_mlp9728_first_blocks(oracle):
+    wl = W.config_mlp9728(64)
+    rep, f = block_teacher_forced(oracle, wl.a, wl.mu, wl.tau, wl.iters, 64, blocks=[0, 1])
+    print(f"mlp9728 b=64: band {rep.band_total} mismatch {rep.band_mismatch} "
+          f"max D rel {rep.d_rel_max:.2e}")
+    assert rep.ok, rep.bad
+    p = os.path.join(os.path.dirname(__file__), "golden", "oracle_energy.json")
+    g = json.load(open(p))["mlp9728_b64"]
+    assert g["k"] == wl.k and g["block"] == 64
+    E = f.energy.cpu().numpy()
+    print(f"  final energy device {E[-1]:.8f} oracle {g['final_energy']:.8f}")
+    assert abs(E[-1] - g["final_energy"]) <= FREE_ENERGY_ATOL
+
+
+def test_block_zero_matrix():
+    A = torch.zeros((96, 80), device="cuda")
+    f = X.decompose(A, 1.0, 0.5, 2, block=16)
+    assert not f.packed_B.any() and not f.packed_C.any() and not f.D.any()
+    assert torch.all(f.energy == 1.0)
+
+
+def test_block_deterministic():
+    A = _dev(W.llm_like(300, 256, 12, n_outliers=3))
+    f1 = X.decompose(A, 1.5, 0.5, 3, block=32)
+    f2 = X.decompose(A, 1.5, 0.5, 3, block=32)
+    for a, b in ((f1.packed_B, f2.packed_B), (f1.packed_C, f2.packed_C), (f1.D, f2.D),
+                 (f1.energy, f2.energy)):
+        assert torch.equal(a, b)
