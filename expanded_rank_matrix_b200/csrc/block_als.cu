@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "umma_layout.cuh"
 
 namespace externd {
 namespace blk {
@@ -54,7 +55,8 @@ __device__ double block_sum_d(double x, double* sh) {
 // ---- setup: R = A, row-energy partials per column chunk, validity -----------
 // Row energies are kept as partials over column chunks of kChunk columns,
 // rhop[chunk][row], summed in chunk order where a full energy is needed.
-constexpr int kChunk = 1024;
+constexpr int kChunk = 1024;  // deflate_kernel assumes 4 x 256 threads
+static_assert(kChunk == 4 * 256, "deflate fill layout");
 __global__ void setup_kernel(const float* __restrict__ A, float* __restrict__ R, int m, int n,
                              const float* __restrict__ w, double* __restrict__ rhop,
                              int* __restrict__ bad) {
@@ -80,36 +82,63 @@ __global__ void setup_kernel(const float* __restrict__ A, float* __restrict__ R,
   }
 }
 
-__global__ void check_w_kernel(const float* __restrict__ w, int n, int* __restrict__ bad) {
+// validity of the weights, and their copy zero padded to npad entries
+__global__ void check_w_kernel(const float* __restrict__ w, int n, int npad,
+                               float* __restrict__ wpad, int* __restrict__ bad) {
   const int j = blockIdx.x * blockDim.x + threadIdx.x;
   if (j < n) {
     const float x = w[j];
     if (!(x > 0.f) || !isfinite(x)) atomicExch(bad, 1);
+    wpad[j] = x;
+  } else if (j < npad) {
+    wpad[j] = 0.f;
   }
 }
 
 // ---- top-bb rows: radix select on the fp64 energy bits, then rank ----------
 // One CTA of 1024 threads.  Also sums the energies in a fixed order (R2) and,
-// on the first block, records it as E0.
+// on the first block, records it as E0.  With `cached` set the m energy keys
+// are kept in dynamic shared memory for the eight radix passes.
 __global__ void __launch_bounds__(1024) select_rows_kernel(const double* __restrict__ rhop,
                                                            int nch, double* __restrict__ rho,
                                                            int m, int bb, int* __restrict__ rows,
                                                            double* __restrict__ scal,
-                                                           int first) {
+                                                           int first, int cached) {
+  extern __shared__ unsigned long long keys_sh[];
   __shared__ unsigned int hist[256];
   __shared__ double sh[32];
   __shared__ unsigned long long s_prefix, s_mask;
   __shared__ int s_remaining;
-  __shared__ int cnt_gt[1024], cnt_eq[1024];
+  __shared__ int cnt_gt[64], cnt_eq[64];
   __shared__ int cand[kMaxB];
   const int tid = threadIdx.x;
   double part = 0.0;
-  for (int i = tid; i < m; i += 1024) {
-    double r = 0.0;
-    for (int c = 0; c < nch; ++c) r += rhop[(size_t)c * m + i];
-    rho[i] = r;
-    part += r;
+  for (int i0 = 0; i0 < m; i0 += 4096) {
+    // four rows per thread per round, every partial load in flight together
+    double r[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int c = 0; c < nch; ++c) {
+      double v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int i = i0 + tid + 1024 * q;
+        v[q] = i < m ? rhop[(size_t)c * m + i] : 0.0;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) r[q] += v[q];
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = i0 + tid + 1024 * q;
+      if (i < m) {
+        rho[i] = r[q];
+        if (cached) keys_sh[i] = (u64)__double_as_longlong(r[q]);
+        part += r[q];
+      }
+    }
   }
+  auto key_of = [&](int i) -> u64 {
+    return cached ? keys_sh[i] : (u64)__double_as_longlong(rho[i]);
+  };
   const double R2 = block_sum_d(part, sh);
   if (tid == 0) {
     scal[0] = R2;
@@ -124,20 +153,43 @@ __global__ void __launch_bounds__(1024) select_rows_kernel(const double* __restr
     __syncthreads();
     const u64 pref = s_prefix, msk = s_mask;
     for (int i = tid; i < m; i += 1024) {
-      const u64 key = (u64)__double_as_longlong(rho[i]);
+      const u64 key = key_of(i);
       if ((key & msk) == pref) atomicAdd(&hist[(key >> shift) & 0xffu], 1u);
     }
     __syncthreads();
-    if (tid == 0) {
-      int rem = s_remaining;
-      int d = 255;
-      for (; d > 0; --d) {
-        if ((int)hist[d] >= rem) break;
-        rem -= (int)hist[d];
+    if (tid < 32) {
+      // lane L owns digits 255 - 8L down to 248 - 8L; the digit sought is the
+      // largest d whose count from the top reaches the rows still needed
+      const int rem = s_remaining;
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        cnt[q] = (int)hist[255 - 8 * tid - q];
+        tot += cnt[q];
       }
-      s_remaining = rem;
-      s_prefix = pref | ((u64)d << shift);
-      s_mask = msk | (0xffull << shift);
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const int excl = incl - tot;
+      // the owner lane: excl < rem <= incl (the last lane takes digit 0 otherwise)
+      const bool own = (excl < rem && rem <= incl) || (tid == 31 && incl < rem);
+      if (own) {
+        int r = rem - excl, dd = 255 - 8 * tid - 7;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (cnt[q] >= r) {
+            dd = 255 - 8 * tid - q;
+            break;
+          }
+          r -= cnt[q];
+        }
+        s_remaining = r;
+        s_prefix = pref | ((u64)dd << shift);
+        s_mask = msk | (0xffull << shift);
+      }
     }
     __syncthreads();
   }
@@ -148,28 +200,50 @@ __global__ void __launch_bounds__(1024) select_rows_kernel(const double* __restr
   const int i0 = min(m, tid * per), i1 = min(m, i0 + per);
   int g = 0, e = 0;
   for (int i = i0; i < i1; ++i) {
-    const u64 key = (u64)__double_as_longlong(rho[i]);
+    const u64 key = key_of(i);
     g += key > kstar;
     e += key == kstar;
   }
-  cnt_gt[tid] = g;
-  cnt_eq[tid] = e;
-  __syncthreads();
-  if (tid == 0) {  // exclusive scans (1024 entries, cheap)
-    int ag = 0, ae = 0;
-    for (int t = 0; t < 1024; ++t) {
-      const int tg = cnt_gt[t], te = cnt_eq[t];
-      cnt_gt[t] = ag;
-      cnt_eq[t] = ae;
-      ag += tg;
-      ae += te;
+  // exclusive scans of both counts in thread order: warp scans, then the
+  // 32 warp totals scanned by warp 0
+  {
+    const int lane = tid & 31, wq = tid >> 5;
+    int ig = g, ie = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int yg = __shfl_up_sync(0xffffffffu, ig, o), ye = __shfl_up_sync(0xffffffffu, ie, o);
+      if (lane >= o) {
+        ig += yg;
+        ie += ye;
+      }
     }
+    if (lane == 31) {
+      cnt_gt[wq] = ig;
+      cnt_eq[wq] = ie;
+    }
+    __syncthreads();
+    if (wq == 0) {
+      int tg = cnt_gt[lane], te = cnt_eq[lane];
+      int sg = tg, se = te;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yg = __shfl_up_sync(0xffffffffu, sg, o), ye = __shfl_up_sync(0xffffffffu, se, o);
+        if (lane >= o) {
+          sg += yg;
+          se += ye;
+        }
+      }
+      cnt_gt[32 + lane] = sg - tg;
+      cnt_eq[32 + lane] = se - te;
+    }
+    __syncthreads();
+    g = cnt_gt[32 + wq] + ig - g;
+    e = cnt_eq[32 + wq] + ie - e;
   }
-  __syncthreads();
-  int pg = cnt_gt[tid], pe = cnt_eq[tid];
+  int pg = g, pe = e;
   const int ngt = bb - need_eq;  // rows strictly above kstar
   for (int i = i0; i < i1; ++i) {
-    const u64 key = (u64)__double_as_longlong(rho[i]);
+    const u64 key = key_of(i);
     if (key > kstar) {
       if (pg < kMaxB) cand[pg] = i;
       ++pg;
@@ -182,11 +256,11 @@ __global__ void __launch_bounds__(1024) select_rows_kernel(const double* __restr
   // order the bb candidates by (energy desc, index asc)
   if (tid < bb) {
     const int me = cand[tid];
-    const double rm = rho[me];
+    const double rm = __longlong_as_double((long long)key_of(me));
     int rank = 0;
     for (int t = 0; t < bb; ++t) {
       const int o = cand[t];
-      const double ro = rho[o];
+      const double ro = __longlong_as_double((long long)key_of(o));
       rank += (ro > rm) || (ro == rm && o < me);
     }
     rows[rank] = me;
@@ -212,9 +286,25 @@ __global__ void vinit_kernel(const float* __restrict__ R, int n, const int* __re
   }
 }
 
+// Writes the tensor-core B chunk of plane word t (entries 32t .. 32t+31): lane
+// holds the plane words of components lane and lane + 32 (zero beyond bb).
+__device__ __forceinline__ void write_bchunk(unsigned char* __restrict__ bop, int t, int lane,
+                                             const uint32_t (&om)[2], const uint32_t (&os)[2]) {
+  unsigned char* chunk = bop + (size_t)t * umma::kBBytes;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int l = lane + 32 * h;
+#pragma unroll
+    for (int kg = 0; kg < 4; ++kg)
+      *(uint4*)(chunk + umma::kmaj_off(l, kg * 8)) =
+          umma::bf16_codes8((om[h] >> (8 * kg)) & 0xffu, (os[h] >> (8 * kg)) & 0xffu);
+  }
+}
+
 // ---- packed planes [bb][2][W] of per-entry 64-bit masks (warp per word) ------
 __global__ void planes_kernel(const u64* __restrict__ Mk, const u64* __restrict__ Sg, int len,
-                              int bb, uint32_t* __restrict__ planes, int W) {
+                              int bb, uint32_t* __restrict__ planes, int W,
+                              unsigned char* __restrict__ bop) {
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= W) return;
@@ -236,6 +326,7 @@ __global__ void planes_kernel(const u64* __restrict__ Mk, const u64* __restrict_
       planes[(size_t)l * 2 * W + W + t] = os[h];
     }
   }
+  if (bop) write_bchunk(bop, t, lane, om, os);
 }
 
 // ---- Gram matrix from packed planes: G[l][l2] = sum_x w_x s_xl s_xl2 --------
@@ -257,12 +348,18 @@ __global__ void gram_kernel(const uint32_t* __restrict__ planes, int W, int bb,
   const uint32_t* m2 = planes + (size_t)l2 * 2 * W;
   double acc = 0.0;
   long long cnt = 0;
-  for (int t = lane; t < W; t += 32) {
-    const uint32_t mm = m1[t] & m2[t];
-    const uint32_t x = m1[W + t] ^ m2[W + t];
-    if (!w) {
+  if (!w) {
+    // unrolled so the plane loads of several words are in flight together
+#pragma unroll 4
+    for (int t = lane; t < W; t += 32) {
+      const uint32_t mm = m1[t] & m2[t];
+      const uint32_t x = m1[W + t] ^ m2[W + t];
       cnt += (long long)__popc(mm & ~x) - (long long)__popc(mm & x);
-    } else {
+    }
+  } else {
+    for (int t = lane; t < W; t += 32) {
+      const uint32_t mm = m1[t] & m2[t];
+      const uint32_t x = m1[W + t] ^ m2[W + t];
       uint32_t bits = mm;
       while (bits) {
         const int b = __ffs(bits) - 1;
@@ -285,41 +382,86 @@ __global__ void gram_kernel(const uint32_t* __restrict__ planes, int W, int bb,
   }
 }
 
-// ---- S = (G + eps I)^-1 by Gauss-Jordan on [G + eps I | I] (SPD, no pivots) --
-// Dynamic shared memory: bb x 2bb doubles + bb doubles.
-__global__ void __launch_bounds__(256) inv_kernel(const double* __restrict__ G, int bb,
-                                                  double* __restrict__ S) {
-  extern __shared__ double ash[];
-  const int w2 = 2 * bb;
-  double* Am = ash;
-  __shared__ double eps;
-  if (threadIdx.x == 0) {
-    double tr = 0.0;
-    for (int l = 0; l < bb; ++l) tr += G[l * bb + l];
-    eps = tr > 0.0 ? 1e-6 * tr / (double)bb : 1.0;
+// ---- in-place Gauss-Jordan inverse of an SPD matrix (no pivoting) ----------
+// The bb x bb matrix (bb <= 64, zero padded to 64 x 64) lives in registers of
+// a 256-thread CTA: warp w holds rows 8w .. 8w+7, lane holds columns lane and
+// lane + 32.  Pivot k: its owner warp publishes row k to shared memory (two
+// alternating buffers, so one barrier per pivot suffices); every thread then
+// forms the scaled pivot row n = a_k / a_kk (n_k = 1 / a_kk) for its columns
+// and updates its rows, a_ij <- a_ij - a_ik n_j for j != k and
+// a_ik <- -a_ik n_k.  After bb pivots the registers hold the inverse.
+__device__ __forceinline__ void gj_inverse(double (&a)[8][2], int bb, double* prow) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  // row 0 is published up front; row k + 1 by its owner right after it has
+  // been updated in step k (selecting a register row by a runtime index
+  // would force the matrix into local memory)
+  if (wid == 0) {
+    prow[lane] = a[0][0];
+    prow[lane + 32] = a[0][1];
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < bb * w2; e += blockDim.x) {
-    const int i = e / w2, j = e - i * w2;
-    Am[e] = j < bb ? G[i * bb + j] + (i == j ? eps : 0.0) : (j - bb == i ? 1.0 : 0.0);
-  }
-  __syncthreads();
-  // thread (row r = tid / 4, column phase cq = tid % 4) -- blockDim.x == 256
-  const int r = threadIdx.x >> 2, cq = threadIdx.x & 3;
   for (int k = 0; k < bb; ++k) {
-    const double inv = 1.0 / Am[k * w2 + k];
-    const double f = (r < bb && r != k) ? Am[r * w2 + k] : 0.0;
     __syncthreads();
-    if (r == k)
-      for (int j = cq; j < w2; j += 4) Am[k * w2 + j] *= inv;
-    __syncthreads();
-    if (r < bb && r != k)
-      for (int j = cq; j < w2; j += 4) Am[r * w2 + j] -= f * Am[k * w2 + j];
-    __syncthreads();
+    const double* pr = prow + (k & 1) * kMaxB;
+    const double p = 1.0 / pr[k];
+    const double n0 = lane == k ? p : pr[lane] * p;
+    const double n1 = lane + 32 == k ? p : pr[lane + 32] * p;
+    const int lk = k & 31;
+    const bool hi = k >= 32;
+    double* nx = prow + ((k + 1) & 1) * kMaxB;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const double f0 = __shfl_sync(0xffffffffu, a[q][0], lk);
+      const double f1 = __shfl_sync(0xffffffffu, a[q][1], lk);
+      const double f = hi ? f1 : f0;
+      if (wid * 8 + q == k) {
+        a[q][0] = n0;
+        a[q][1] = n1;
+      } else {
+        a[q][0] = (lane == k ? 0.0 : a[q][0]) - f * n0;
+        a[q][1] = (lane + 32 == k ? 0.0 : a[q][1]) - f * n1;
+      }
+      if (wid * 8 + q == k + 1) {
+        nx[lane] = a[q][0];
+        nx[lane + 32] = a[q][1];
+      }
+    }
   }
-  for (int e = threadIdx.x; e < bb * bb; e += blockDim.x) {
-    const int i = e / bb, j = e - i * bb;
-    S[e] = Am[i * w2 + bb + j];
+  __syncthreads();
+}
+
+// S = (G + eps I)^-1 with eps = 1e-6 tr(G) / bb (1 when the trace is 0).
+__global__ void __launch_bounds__(256, 1) inv_kernel(const double* __restrict__ G, int bb,
+                                                  double* __restrict__ S) {
+  __shared__ double prow[2 * kMaxB];
+  __shared__ double eps;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (wid == 0) {
+    double t = (lane < bb ? G[lane * bb + lane] : 0.0) +
+               (lane + 32 < bb ? G[(lane + 32) * bb + lane + 32] : 0.0);
+    // fixed-order tree over the 64 diagonal entries
+    t = warp_sum(t);
+    if (lane == 0) eps = t > 0.0 ? 1e-6 * t / (double)bb : 1.0;
+  }
+  __syncthreads();
+  double a[8][2];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int i = wid * 8 + q;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = lane + 32 * h;
+      a[q][h] = (i < bb && j < bb) ? G[i * bb + j] + (i == j ? eps : 0.0) : 0.0;
+    }
+  }
+  gj_inverse(a, bb, prow);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int i = wid * 8 + q;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = lane + 32 * h;
+      if (i < bb && j < bb) S[i * bb + j] = a[q][h];
+    }
   }
 }
 
@@ -428,72 +570,224 @@ __global__ void __launch_bounds__(256) rtu_kernel(const float* __restrict__ R, i
   }
 }
 
-// ---- targets: T[x][l] = sum_l2 (sum_s Xp[s][x][l2]) S[l2][l] (fp64), and
-// per-CTA column sums of squares.  16 rows per CTA, 4 per step.
-constexpr int kTgtRows = 16;
-__global__ void __launch_bounds__(256) target_kernel(const float* __restrict__ Xp, int splits,
-                                                     int rows, int bb, const double* __restrict__ S,
-                                                     double* __restrict__ T,
-                                                     double* __restrict__ colss) {
-  __shared__ double Ss[kMaxB * kMaxB];
-  __shared__ double xr[4][kMaxB];
-  __shared__ double part[4][kMaxB];
-  for (int p = threadIdx.x; p < bb * bb; p += 256) Ss[p] = S[p];
-  const int l = threadIdx.x & 63, rr = threadIdx.x >> 6;
-  double cs = 0.0;
-  const int x0 = blockIdx.x * kTgtRows;
-  for (int base = x0; base < min(rows, x0 + kTgtRows); base += 4) {
-    __syncthreads();
-    {
-      const int x = base + rr;
-      if (l < bb) {
-        double s = 0.0;
-        if (x < rows)
-          for (int sp = 0; sp < splits; ++sp) s += (double)Xp[((size_t)sp * rows + x) * bb + l];
-        xr[rr][l] = s;
+// ---- targets: T[x][l] = sum_l2 (sum_s Xp[s][x][l2]) S[l2][l] (fp64) ----------
+// 64 rows per CTA, two CTAs per SM (one wave for up to 2 x SMs x 64 rows).
+// The split-K partials are summed (split order, fp64) into a transposed tile
+// Xt[l2][row] in shared memory next to S -- each thread loads 4 consecutive
+// columns of 4 rows, float4 per split, all splits in flight (NS >= splits is
+// a compile-time bound).  Thread (rg, cg) then forms the 4 x 4 block rows
+// 4rg.., columns 4cg.. of T: 16 independent fp64 chains per thread.  Each CTA
+// writes its column sums of squares; the last CTA to finish (ticket counter)
+// sums those partials in CTA order and writes the column thresholds
+// thr[l] = tau * rms(T[:, l]), then rearms the counter.  With Xout set, the
+// split-summed X (rows x bb, fp64) is stored as well.
+constexpr int kTgtRows2 = 64;  // rows per CTA of target_kernel
+constexpr int kMaxSplits = 16; // split-K partials per contraction
+constexpr int kXs = kTgtRows2 + 2;  // padded row of the transposed tile (16-byte aligned)
+template <int NS>
+__global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict__ Xp, int splits,
+                                                        int rows, int bb,
+                                                        const double* __restrict__ S, double tau,
+                                                        double* __restrict__ T,
+                                                        double* __restrict__ colss,
+                                                        unsigned* __restrict__ ticket,
+                                                        double* __restrict__ thr,
+                                                        double* __restrict__ Xout) {
+  extern __shared__ __align__(16) double tsh[];
+  double* Ss = tsh;                                                 // [64][64]: S[l2][l]
+  double* Xt = tsh + kMaxB * kMaxB;                                 // [64][kXs]
+  double (*part)[kMaxB] = (double (*)[kMaxB])(Xt + kMaxB * kXs);    // [16][64]
+  __shared__ bool last;
+  const int tid = threadIdx.x;
+  const int x0 = blockIdx.x * kTgtRows2;
+  {
+    double sv[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int p = tid + 256 * q, l2 = p >> 6, lc = p & 63;
+      sv[q] = (l2 < bb && lc < bb) ? __ldg(S + l2 * bb + lc) : 0.0;
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) Ss[tid + 256 * q] = sv[q];
+  }
+  {
+    // thread: columns lq .. lq+3 (lq = 4 (tid % 16)), rows tid / 16 + 16 h
+    const int lq = (tid & 15) * 4, rr = tid >> 4;
+    const size_t sstride = (size_t)rows * bb;
+    const bool vec = (bb & 3) == 0;
+    constexpr int RPR = NS > 8 ? 1 : 2;  // rows per round: at most 64 floats in flight
+#pragma unroll 1
+    for (int h0 = 0; h0 < 4; h0 += RPR) {
+      float4 v[RPR][NS];
+#pragma unroll
+      for (int h = 0; h < RPR; ++h) {
+        const int x = x0 + rr + 16 * (h0 + h);
+        const bool ok = x < rows && lq < bb;
+        const float* src = Xp + (size_t)(ok ? x : 0) * bb + (ok ? lq : 0);
+#pragma unroll
+        for (int sp = 0; sp < NS; ++sp) {
+          float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (ok && sp < splits) {
+            const float* q = src + sp * sstride;
+            if (vec) {
+              t = __ldg((const float4*)q);
+            } else {
+              t.x = __ldg(q);
+              if (lq + 1 < bb) t.y = __ldg(q + 1);
+              if (lq + 2 < bb) t.z = __ldg(q + 2);
+              if (lq + 3 < bb) t.w = __ldg(q + 3);
+            }
+          }
+          v[h][sp] = t;
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < RPR; ++h) {
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+#pragma unroll
+        for (int sp = 0; sp < NS; ++sp)
+          if (sp < splits) {
+            s0 += (double)v[h][sp].x;
+            s1 += (double)v[h][sp].y;
+            s2 += (double)v[h][sp].z;
+            s3 += (double)v[h][sp].w;
+          }
+        const int r = rr + 16 * (h0 + h);
+        Xt[(lq + 0) * kXs + r] = s0;
+        Xt[(lq + 1) * kXs + r] = s1;
+        Xt[(lq + 2) * kXs + r] = s2;
+        Xt[(lq + 3) * kXs + r] = s3;
+        const int x = x0 + r;
+        if (Xout && x < rows) {
+          const double sx[4] = {s0, s1, s2, s3};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (lq + j < bb) Xout[(size_t)x * bb + lq + j] = sx[j];
+        }
       }
     }
-    __syncthreads();
-    const int x = base + rr;
-    if (x < rows && l < bb) {
-      double t = 0.0;
-      for (int l2 = 0; l2 < bb; ++l2) t += xr[rr][l2] * Ss[l2 * bb + l];
-      T[(size_t)x * bb + l] = t;
-      cs += t * t;
+  }
+  __syncthreads();
+  const int rg = tid >> 4, cg = tid & 15;
+  double acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+#pragma unroll 2
+  for (int l2 = 0; l2 < bb; ++l2) {
+    const double2 xa = *(const double2*)(Xt + l2 * kXs + 4 * rg);
+    const double2 xb = *(const double2*)(Xt + l2 * kXs + 4 * rg + 2);
+    const double2 sa = *(const double2*)(Ss + l2 * kMaxB + 4 * cg);
+    const double2 sb = *(const double2*)(Ss + l2 * kMaxB + 4 * cg + 2);
+    const double xv[4] = {xa.x, xa.y, xb.x, xb.y}, svv[4] = {sa.x, sa.y, sb.x, sb.y};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += xv[i] * svv[j];
+  }
+  double cs[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int x = x0 + 4 * rg + i;
+    if (x < rows) {
+      if (bb == kMaxB) {
+        *(double2*)(T + (size_t)x * bb + 4 * cg) = make_double2(acc[i][0], acc[i][1]);
+        *(double2*)(T + (size_t)x * bb + 4 * cg + 2) = make_double2(acc[i][2], acc[i][3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (4 * cg + j < bb) T[(size_t)x * bb + 4 * cg + j] = acc[i][j];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cs[j] += acc[i][j] * acc[i][j];
     }
   }
-  part[rr][l] = cs;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) part[rg][4 * cg + j] = cs[j];
   __syncthreads();
-  if (rr == 0 && l < bb)
-    colss[(size_t)blockIdx.x * bb + l] = ((part[0][l] + part[1][l]) + part[2][l]) + part[3][l];
-}
-
-// ---- thresholds per column; 64-bit masks per entry and packed planes -------
-// One warp per 32 entries (one plane word).
-__global__ void tern_kernel(const double* __restrict__ T, int rows, int bb,
-                            const double* __restrict__ colss, int nparts, double tau,
-                            u64* __restrict__ Mk, u64* __restrict__ Sg,
-                            uint32_t* __restrict__ planes, int W) {
-  __shared__ double thr[kMaxB];
-  if (threadIdx.x < bb) {
-    double s = 0.0;
-    for (int b = 0; b < nparts; ++b) s += colss[(size_t)b * bb + threadIdx.x];
-    thr[threadIdx.x] = tau * sqrt(s / (double)rows);
+  if (tid < kMaxB) {
+    double c = 0.0;
+    for (int g = 0; g < 16; ++g) c += part[g][tid];
+    if (tid < bb) colss[(size_t)blockIdx.x * bb + tid] = c;
   }
   __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  {
+    // thread (q, l) sums the partials of CTAs b = q mod 4 in CTA order, eight
+    // loads in flight; the four sums are then added in q order
+    const int l = tid & 63, q = tid >> 6;
+    double c = 0.0;
+    if (l < bb) {
+      const unsigned nb = gridDim.x;
+      unsigned b = q;
+      for (; b + 28 < nb; b += 32) {
+        double v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(colss + (size_t)(b + 4 * u) * bb + l);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) c += v[u];
+      }
+      for (; b < nb; b += 4) c += __ldcg(colss + (size_t)b * bb + l);
+    }
+    part[q][l] = c;
+    __syncthreads();
+    if (tid < bb) {
+      const double t4 = ((part[0][tid] + part[1][tid]) + part[2][tid]) + part[3][tid];
+      thr[tid] = tau * sqrt(t4 / (double)rows);
+    }
+  }
+  if (tid == 0) *ticket = 0u;
+}
+constexpr size_t kTgtSmem = sizeof(double) * (kMaxB * kMaxB + kMaxB * kXs + 16 * kMaxB);
+// the target kernel instantiated for a split-count bound
+typedef void (*TargetFn)(const float*, int, int, int, const double*, double, double*, double*,
+                         unsigned*, double*, double*);
+inline TargetFn target_for(int splits) {
+  if (splits <= 1) return target_kernel<1>;
+  if (splits <= 2) return target_kernel<2>;
+  if (splits <= 4) return target_kernel<4>;
+  if (splits <= 8) return target_kernel<8>;
+  return target_kernel<16>;
+}
+
+// ---- ternary codes: 64-bit masks per entry and packed planes -----------------
+// One warp per 32 entries (one plane word): lanes read the entry's T row
+// (coalesced) and ballot the threshold tests, so lane r ends up holding the
+// masks of entry r; 64 more ballots per warp transpose them into planes.
+__global__ void tern_kernel(const double* __restrict__ T, int rows, int bb,
+                            const double* __restrict__ thr, u64* __restrict__ Mk,
+                            u64* __restrict__ Sg, uint32_t* __restrict__ planes, int W,
+                            unsigned char* __restrict__ bop) {
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= W) return;
-  const int x = t * 32 + lane;
+  const double th0 = lane < bb ? thr[lane] : 0.0, th1 = lane + 32 < bb ? thr[lane + 32] : 0.0;
   u64 mk = 0ull, sg = 0ull;
-  if (x < rows)
-    for (int l = 0; l < bb; ++l) {
-      const double v = T[(size_t)x * bb + l];
-      if (fabs(v) > thr[l]) {
-        mk |= 1ull << l;
-        if (v < 0.0) sg |= 1ull << l;
-      }
+#pragma unroll 8
+  for (int r = 0; r < 32; ++r) {
+    const int x = t * 32 + r;
+    double v0 = 0.0, v1 = 0.0;
+    if (x < rows) {
+      if (lane < bb) v0 = T[(size_t)x * bb + lane];
+      if (lane + 32 < bb) v1 = T[(size_t)x * bb + lane + 32];
     }
+    const bool a0 = lane < bb && fabs(v0) > th0, a1 = lane + 32 < bb && fabs(v1) > th1;
+    const uint32_t m0 = __ballot_sync(0xffffffffu, a0), m1 = __ballot_sync(0xffffffffu, a1);
+    const uint32_t s0 = __ballot_sync(0xffffffffu, a0 && v0 < 0.0);
+    const uint32_t s1 = __ballot_sync(0xffffffffu, a1 && v1 < 0.0);
+    if (lane == r) {
+      mk = (u64)m0 | ((u64)m1 << 32);
+      sg = (u64)s0 | ((u64)s1 << 32);
+    }
+  }
+  const int x = t * 32 + lane;
   if (x < rows) {
     Mk[x] = mk;
     Sg[x] = sg;
@@ -514,27 +808,32 @@ __global__ void tern_kernel(const double* __restrict__ T, int rows, int bb,
       planes[(size_t)l * 2 * W + W + t] = os[h];
     }
   }
+  if (bop) write_bchunk(bop, t, lane, om, os);
 }
 
-// ---- r_l = u_l^T R W v_l = sum_j (sum_s Qp[s][j][l]) w_j s_jl, per-CTA partials
-__global__ void __launch_bounds__(256) rpart_kernel(const float* __restrict__ Qp, int splits, int n,
-                                                    int bb, const u64* __restrict__ Vm,
+// ---- r_l = u_l^T R W v_l = sum_j Q[j][l] w_j s_jl, per-CTA partials (64 rows)
+// Q = R^T U, split-summed in fp64 by the last V-step target pass.
+__global__ void __launch_bounds__(256) rpart_kernel(const double* __restrict__ Q, int n, int bb,
+                                                    const u64* __restrict__ Vm,
                                                     const u64* __restrict__ Vs,
                                                     const float* __restrict__ w,
                                                     double* __restrict__ rp) {
   __shared__ double part[4][kMaxB];
   const int l = threadIdx.x & 63, rr = threadIdx.x >> 6;
-  const int x0 = blockIdx.x * kTgtRows;
+  const int x0 = blockIdx.x * kTgtRows2;
   double acc = 0.0;
-  if (l < bb)
-    for (int j = x0 + rr; j < min(n, x0 + kTgtRows); j += 4) {
-      const u64 mm = Vm[j];
-      if (!((mm >> l) & 1ull)) continue;
-      double q = 0.0;
-      for (int sp = 0; sp < splits; ++sp) q += (double)Qp[((size_t)sp * n + j) * bb + l];
-      const double wj = w ? (double)w[j] : 1.0;
-      acc += (((Vs[j] >> l) & 1ull) ? -q : q) * wj;
+  if (l < bb) {
+#pragma unroll 4
+    for (int t = 0; t < kTgtRows2 / 4; ++t) {
+      const int j = x0 + rr + 4 * t;
+      if (j < n) {
+        const u64 mm = Vm[j];
+        const double q = Q[(size_t)j * bb + l];
+        const double wj = w ? (double)w[j] : 1.0;
+        if ((mm >> l) & 1ull) acc += (((Vs[j] >> l) & 1ull) ? -q : q) * wj;
+      }
     }
+  }
   part[rr][l] = acc;
   __syncthreads();
   if (rr == 0 && l < bb)
@@ -542,68 +841,76 @@ __global__ void __launch_bounds__(256) rpart_kernel(const float* __restrict__ Qp
 }
 
 // ---- joint scales, closed-form energies ---------------------------------------
-// r_l = sum_j (sum_s Qp[s][j][l]) w_j s_jl; G = GU o GV; active-set solve.
-__global__ void __launch_bounds__(256) dsolve_kernel(const double* __restrict__ GU,
+// r_l = sum_j (sum_s Qp[s][j][l]) w_j s_jl; G = GU o GV; the active set (l
+// with u_l != 0 and v_l != 0) solves (G_AA + eps I) d_A = r_A through the
+// register Gauss-Jordan inverse; inactive scales are 0.
+__global__ void __launch_bounds__(256, 1) dsolve_kernel(const double* __restrict__ GU,
                                                      const double* __restrict__ GV,
                                                      const double* __restrict__ rp, int rparts,
                                                      int bb, const double* __restrict__ scal,
                                                      int c0, float* __restrict__ D,
                                                      double* __restrict__ energy,
                                                      float* __restrict__ dblk) {
-  extern __shared__ double dsh[];
-  double* G = dsh;                        // bb x bb, (U^T U) o (V^T W V)
-  double* Am = dsh + (size_t)bb * bb;      // active system, A x (A+1)
-  __shared__ double r[kMaxB], fcol[kMaxB];
+  __shared__ double G[kMaxB * kMaxB];
+  __shared__ double r[kMaxB], ra[kMaxB], fcol[kMaxB], prow[2 * kMaxB];
   __shared__ float dl[kMaxB];
   __shared__ int act[kMaxB];
   __shared__ int na;
   __shared__ double eps;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (threadIdx.x < bb) {
     double s = 0.0;
+#pragma unroll 8
     for (int b = 0; b < rparts; ++b) s += rp[(size_t)b * bb + threadIdx.x];
     r[threadIdx.x] = s;
     dl[threadIdx.x] = 0.f;
   }
   for (int p = threadIdx.x; p < bb * bb; p += blockDim.x) G[p] = GU[p] * GV[p];
   __syncthreads();
-  if (threadIdx.x == 0) {
-    double tr = 0.0;
-    for (int l = 0; l < bb; ++l) tr += G[l * bb + l];
-    eps = tr > 0.0 ? 1e-6 * tr / (double)bb : 1.0;
-    int c = 0;
-    for (int l = 0; l < bb; ++l)
-      if (GU[l * bb + l] > 0.0 && GV[l * bb + l] > 0.0) act[c++] = l;
-    na = c;
-  }
-  __syncthreads();
-  const int A = na, w2 = A + 1;
-  for (int e = threadIdx.x; e < A * w2; e += blockDim.x) {
-    const int a = e / w2, c = e - a * w2;
-    Am[e] = c < A ? G[act[a] * bb + act[c]] + (a == c ? eps : 0.0) : r[act[a]];
-  }
-  __syncthreads();
-  {
-    const int rr = threadIdx.x >> 2, cq = threadIdx.x & 3;
-    for (int k = 0; k < A; ++k) {
-      const double inv = 1.0 / Am[k * w2 + k];
-      const double f = (rr < A && rr != k) ? Am[rr * w2 + k] : 0.0;
-      __syncthreads();
-      if (rr == k)
-        for (int j = cq; j < w2; j += 4) Am[k * w2 + j] *= inv;
-      __syncthreads();
-      if (rr < A && rr != k)
-        for (int j = cq; j < w2; j += 4) Am[rr * w2 + j] -= f * Am[k * w2 + j];
-      __syncthreads();
+  if (wid == 0) {
+    double t = (lane < bb ? G[lane * bb + lane] : 0.0) +
+               (lane + 32 < bb ? G[(lane + 32) * bb + lane + 32] : 0.0);
+    t = warp_sum(t);
+    const bool a0 = lane < bb && GU[lane * bb + lane] > 0.0 && GV[lane * bb + lane] > 0.0;
+    const bool a1 = lane + 32 < bb && GU[(lane + 32) * bb + lane + 32] > 0.0 &&
+                    GV[(lane + 32) * bb + lane + 32] > 0.0;
+    const unsigned b0 = __ballot_sync(0xffffffffu, a0), b1 = __ballot_sync(0xffffffffu, a1);
+    const unsigned below = (1u << lane) - 1u;
+    if (a0) act[__popc(b0 & below)] = lane;
+    if (a1) act[__popc(b0) + __popc(b1 & below)] = lane + 32;
+    if (lane == 0) {
+      eps = t > 0.0 ? 1e-6 * t / (double)bb : 1.0;
+      na = __popc(b0) + __popc(b1);
     }
   }
-  for (int a = threadIdx.x; a < A; a += blockDim.x) dl[act[a]] = (float)Am[a * w2 + A];
+  __syncthreads();
+  const int A = na;
+  if (threadIdx.x < A) ra[threadIdx.x] = r[act[threadIdx.x]];
+  double a[8][2];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int i = wid * 8 + q;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = lane + 32 * h;
+      a[q][h] = (i < A && j < A) ? G[act[i] * bb + act[j]] + (i == j ? eps : 0.0) : 0.0;
+    }
+  }
+  gj_inverse(a, A, prow);  // ends with a barrier, which also publishes ra
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int i = wid * 8 + q;
+    double t = (lane < A ? a[q][0] * ra[lane] : 0.0) + (lane + 32 < A ? a[q][1] * ra[lane + 32] : 0.0);
+    t = warp_sum(t);
+    if (lane == 0 && i < A) dl[act[i]] = (float)t;
+  }
   __syncthreads();
   // energy after component c0 + l: |R|^2 - 2 sum_{a<=l} d_a r_a + sum_{a,c<=l} d_a d_c G_ac,
   // accumulated over l: inc_l = -2 d_l r_l + d_l^2 G_ll + 2 d_l sum_{a<l} d_a G_al
   if (threadIdx.x < bb) {
     const int l = threadIdx.x;
     double h = 0.0;
-    for (int a = 0; a < l; ++a) h += (double)dl[a] * G[a * bb + l];
+    for (int q = 0; q < l; ++q) h += (double)dl[q] * G[q * bb + l];
     const double dd = (double)dl[l];
     fcol[l] = -2.0 * dd * r[l] + dd * dd * G[l * bb + l] + 2.0 * dd * h;
     D[c0 + l] = dl[l];
@@ -621,8 +928,13 @@ __global__ void __launch_bounds__(256) dsolve_kernel(const double* __restrict__ 
 }
 
 // ---- ordered block deflation + next block's row-energy partials ------------
-// CTA = 8 warps = 8 rows x one column chunk; V masks of the chunk in shared
-// memory; each lane advances 4 entries' ordered add/subtract chains together.
+// CTA = 8 warps x 2 rows each, over one chunk of kChunk columns whose V masks
+// sit in shared memory.  Row i's active components (u_il != 0) form a list
+// in ascending l with signed scales du_l = u_il d_l.  Each lane holds 4
+// entries x_j and, per entry, which active components meet v_jl = +1 (mask P)
+// or v_jl = -1 (mask N), split into 32-bit halves; the list is walked once
+// per half, so one component costs a bit test and a predicated fp32 add or
+// subtract per entry: x_j <- x_j - du_l (P) or x_j + du_l (N), in ascending l.
 __global__ void __launch_bounds__(256) deflate_kernel(float* __restrict__ R, int m, int n,
                                                       const u64* __restrict__ Um,
                                                       const u64* __restrict__ Us,
@@ -633,70 +945,100 @@ __global__ void __launch_bounds__(256) deflate_kernel(float* __restrict__ R, int
                                                       double* __restrict__ rhop) {
   __shared__ u64 vm[kChunk], vs[kChunk];
   __shared__ float d[kMaxB];
-  const int ch = blockIdx.y, j0 = ch * kChunk, j1 = min(n, j0 + kChunk);
-  for (int j = threadIdx.x; j < j1 - j0; j += blockDim.x) {
-    vm[j] = Vm[j0 + j];
-    vs[j] = Vs[j0 + j];
+  __shared__ int ls_s[8][kMaxB];
+  __shared__ float du_s[8][kMaxB];
+  const int ch = blockIdx.y, j0 = ch * kChunk, j1 = min(n, j0 + kChunk), nj = j1 - j0;
+  {
+    // kChunk / 256 = 4 entries per thread, all loads issued before the stores
+    u64 a[4], b[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = threadIdx.x + 256 * q;
+      a[q] = j < nj ? Vm[j0 + j] : 0ull;
+      b[q] = j < nj ? Vs[j0 + j] : 0ull;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      vm[threadIdx.x + 256 * q] = a[q];
+      vs[threadIdx.x + 256 * q] = b[q];
+    }
   }
   if (threadIdx.x < kMaxB) d[threadIdx.x] = dblk[threadIdx.x];
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int i = blockIdx.x * 8 + wid;
-  if (i >= m) return;
-  const u64 um = Um[i];
-  if (um == 0ull) return;  // untouched row: R and its energy partials stay
-  const u64 us = Us[i];
-  // signed scales of the row's components, in ascending component order
-  // (per-warp lists in shared memory; every lane computes the same list)
-  __shared__ int ls_s[8][kMaxB];
-  __shared__ float du_s[8][kMaxB];
   int* ls = ls_s[wid];
   float* dus = du_s[wid];
-  int nl = 0;
-  for (u64 bits = um; bits; bits &= bits - 1ull) {
-    const int l = __ffsll((long long)bits) - 1;
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = blockIdx.x * 16 + wid * 2 + rr;
+    if (i >= m) break;
+    const u64 um = Um[i];
+    if (um == 0ull) continue;  // untouched row: R and its energy partials stay
+    const u64 us = Us[i];
+    // active components in ascending order; nlo of them below 32
+    __syncwarp();
+    const int nl = __popcll(um), nlo = __popc((uint32_t)um);
     if (lane == 0) {
-      ls[nl] = l;
-      dus[nl] = ((us >> l) & 1ull) ? -d[l] : d[l];
+      int c = 0;
+      for (u64 bits = um; bits; bits &= bits - 1ull, ++c) {
+        const int l = __ffsll((long long)bits) - 1;
+        ls[c] = l;
+        dus[c] = ((us >> l) & 1ull) ? -d[l] : d[l];
+      }
     }
-    ++nl;
-  }
-  __syncwarp();
-  float* row = R + (size_t)i * n;
-  double s = 0.0;
-  for (int jb = lane; jb < j1 - j0; jb += 128) {
-    float x[4];
-    u64 m4[4], s4[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = jb + 32 * e;
-      const bool ok = j < j1 - j0;
-      x[e] = ok ? row[j0 + j] : 0.f;
-      m4[e] = ok ? vm[j] : 0ull;
-      s4[e] = ok ? vs[j] : 0ull;
-    }
-    for (int t = 0; t < nl; ++t) {  // same trip count on every lane: no divergence
-      const int l = ls[t];
-      const float du = dus[t];
+    __syncwarp();
+    float* row = R + (size_t)i * n + j0;
+    double s = 0.0;
+    for (int jw = 0; jw < nj; jw += 128) {  // warp-uniform trip count (warp votes inside)
+      const int jb = jw + lane;
+      float x[4];
+      uint32_t plo[4], phi[4], nlo_[4], nhi[4];
+      bool any = false;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float sd = ((s4[e] >> l) & 1ull) ? -du : du;
-        const float y = __fsub_rn(x[e], sd);
-        x[e] = ((m4[e] >> l) & 1ull) ? y : x[e];
+        const int j = jb + 32 * e;
+        const bool ok = j < nj;
+        x[e] = ok ? row[j] : 0.f;
+        const u64 mm = ok ? vm[j] & um : 0ull, sg = ok ? vs[j] : 0ull;
+        const u64 P = mm & ~sg, N = mm & sg;
+        plo[e] = (uint32_t)P;
+        phi[e] = (uint32_t)(P >> 32);
+        nlo_[e] = (uint32_t)N;
+        nhi[e] = (uint32_t)(N >> 32);
+        any |= mm != 0ull;
       }
-    }
+      if (__any_sync(0xffffffffu, any)) {
+        for (int t = 0; t < nlo; ++t) {  // components 0..31: same trip count on every lane
+          const uint32_t bit = 1u << ls[t];
+          const float du = dus[t];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = jb + 32 * e;
-      if (j < j1 - j0) {
-        if ((um & m4[e]) != 0ull) row[j0 + j] = x[e];
-        const double wj = w ? (double)w[j0 + j] : 1.0;
-        s += wj * (double)x[e] * (double)x[e];
+          for (int e = 0; e < 4; ++e) {
+            if (plo[e] & bit) x[e] = __fsub_rn(x[e], du);
+            if (nlo_[e] & bit) x[e] = __fadd_rn(x[e], du);
+          }
+        }
+        for (int t = nlo; t < nl; ++t) {  // components 32..63
+          const uint32_t bit = 1u << (ls[t] - 32);
+          const float du = dus[t];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if (phi[e] & bit) x[e] = __fsub_rn(x[e], du);
+            if (nhi[e] & bit) x[e] = __fadd_rn(x[e], du);
+          }
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = jb + 32 * e;
+        if (j < nj) {
+          if ((plo[e] | phi[e] | nlo_[e] | nhi[e]) != 0u) row[j] = x[e];
+          const double wj = w ? (double)w[j0 + j] : 1.0;
+          s += wj * (double)x[e] * (double)x[e];
+        }
       }
     }
+    s = warp_sum(s);
+    if (lane == 0) rhop[(size_t)ch * m + i] = s;
   }
-  s = warp_sum(s);
-  if (lane == 0) rhop[(size_t)ch * m + i] = s;
 }
 
 __global__ void set_status_kernel(const int* __restrict__ bad, int* __restrict__ status) {
@@ -720,13 +1062,14 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
   const int tileR = tc ? 128 : kTile, kq = 32;
   // split-K factors so each contraction has about two CTAs per SM
   const int tiles_m = (m + tileR - 1) / tileR, tiles_n = (n + tileR - 1) / tileR;
-  int splitP = std::max(1, std::min((2 * nsm + tiles_m - 1) / tiles_m, (n + kq - 1) / kq));
-  int splitQ = std::max(1, std::min((2 * nsm + tiles_n - 1) / tiles_n, (m + kq - 1) / kq));
+  // (at most two CTAs per SM in total, so a contraction runs in one wave)
+  int splitP = std::max(1, std::min({2 * nsm / tiles_m, (n + kq - 1) / kq, kMaxSplits}));
+  int splitQ = std::max(1, std::min({2 * nsm / tiles_n, (m + kq - 1) / kq, kMaxSplits}));
   const int klenP = ((n + splitP - 1) / splitP + kq - 1) / kq * kq;
   const int klenQ = ((m + splitQ - 1) / splitQ + kq - 1) / kq * kq;
   splitP = (n + klenP - 1) / klenP;
   splitQ = (m + klenQ - 1) / klenQ;
-  const int tgtU = (m + kTgtRows - 1) / kTgtRows, tgtV = (n + kTgtRows - 1) / kTgtRows;
+  const int tgtU = (m + kTgtRows2 - 1) / kTgtRows2, tgtV = (n + kTgtRows2 - 1) / kTgtRows2;
   const int nch = (n + kChunk - 1) / kChunk;
   const int mx = std::max(m, n);
   const int Wm = (m + 31) / 32, Wn = (n + 31) / 32;
@@ -748,6 +1091,11 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
   const size_t oT = take(sizeof(double) * (size_t)mx * b);
   const size_t oCs = take(sizeof(double) * (size_t)std::max(tgtU, tgtV) * b);
   const size_t oRp = take(sizeof(double) * (size_t)tgtV * b);
+  const size_t oQs = take(sizeof(double) * (size_t)n * b);
+  const size_t oThr = take(sizeof(double) * kMaxB);
+  const size_t oBopU = take((size_t)Wm * umma::kBBytes), oBopV = take((size_t)Wn * umma::kBBytes);
+  const size_t oWpad = take(sizeof(float) * (size_t)Wn * 32);
+  const size_t oTick = take(sizeof(unsigned));
   const size_t oSV = take(sizeof(double) * b * b), oSU = take(sizeof(double) * b * b);
   const size_t oGU = take(sizeof(double) * b * b), oGV = take(sizeof(double) * b * b);
   const size_t oScal = take(sizeof(double) * 4);
@@ -775,20 +1123,40 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
   double* scal = (double*)(base + oScal);
   float* dblk = (float*)(base + oD);
   int* bad = (int*)(base + oBad);
+  double* thr = (double*)(base + oThr);
+  double* Qs = (double*)(base + oQs);
+  unsigned char* BopU = tc ? (unsigned char*)(base + oBopU) : nullptr;
+  unsigned char* BopV = tc ? (unsigned char*)(base + oBopV) : nullptr;
+  float* wpad = (float*)(base + oWpad);
+  unsigned* tick = (unsigned*)(base + oTick);
   const double tau = (double)h.tau;
   int rc = EXTERND_OK;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  if (cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    if (side) cudaStreamDestroy(side);
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    cudaFreeAsync(ws, st);
+    return EXTERND_ERR_CUDA;
+  }
+  const TargetFn tgtP = target_for(splitP), tgtQ = target_for(splitQ);
+  cudaFuncSetAttribute(tgtP, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgtSmem);
+  cudaFuncSetAttribute(tgtQ, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgtSmem);
+  // the row-energy keys of the radix select stay in shared memory when they fit
+  const size_t sel_smem = (size_t)m * sizeof(u64) <= 160 * 1024 ? (size_t)m * sizeof(u64) : 0;
+  if (sel_smem > 0)
+    cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem);
   auto chk = [&]() {
     if (rc == EXTERND_OK && cudaGetLastError() != cudaSuccess) rc = EXTERND_ERR_CUDA;
   };
-  const size_t ism = sizeof(double) * ((size_t)b * 2 * b + b);
-  const size_t dsm = sizeof(double) * ((size_t)b * b + (size_t)b * (b + 1));
-  if (ism > 48 * 1024) cudaFuncSetAttribute(inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ism);
-  if (dsm > 48 * 1024)
-    cudaFuncSetAttribute(dsolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm);
   cudaMemsetAsync(bad, 0, sizeof(int), st);
+  cudaMemsetAsync(tick, 0, sizeof(unsigned), st);
   cudaMemsetAsync(dblk, 0, sizeof(float) * kMaxB, st);
   setup_kernel<<<dim3((m * 32 + 255) / 256, nch), 256, 0, st>>>(h.A, R, m, n, h.w, rhop, bad);
-  if (h.w) check_w_kernel<<<(n + 255) / 256, 256, 0, st>>>(h.w, n, bad);
+  if (h.w) check_w_kernel<<<(Wn * 32 + 255) / 256, 256, 0, st>>>(h.w, n, Wn * 32, wpad, bad);
   chk();
   // trace record of a block: V0, then U_t and V_t per iteration (mask words
   // then sign words); plus the start rows
@@ -808,33 +1176,46 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
       cudaMemcpyAsync(dst, mk, sizeof(u64) * len, cudaMemcpyDeviceToDevice, st);
       cudaMemcpyAsync(dst + len, sg, sizeof(u64) * len, cudaMemcpyDeviceToDevice, st);
     };
-    select_rows_kernel<<<1, 1024, 0, st>>>(rhop, nch, rho, m, bb, rows, scal, c0 == 0);
+    select_rows_kernel<<<1, 1024, sel_smem, st>>>(rhop, nch, rho, m, bb, rows, scal, c0 == 0,
+                                                  sel_smem > 0);
     cudaMemsetAsync(Vm, 0, sizeof(u64) * n, st);
     cudaMemsetAsync(Vs, 0, sizeof(u64) * n, st);
     vinit_kernel<<<bb, 256, 0, st>>>(R, n, rows, tau, Vm, Vs);
-    planes_kernel<<<(Wn * 32 + 255) / 256, 256, 0, st>>>(Vm, Vs, n, bb, pC, Wn);
+    planes_kernel<<<(Wn * 32 + 255) / 256, 256, 0, st>>>(Vm, Vs, n, bb, pC, Wn, BopV);
     if (tr) {
       cudaMemcpyAsync(h.trace_rows + (size_t)tslot * b, rows, sizeof(int) * bb,
                       cudaMemcpyDeviceToDevice, st);
       record(tr, Vm, Vs, n);
     }
     for (int it = 0; it < h.iters; ++it) {
-      gram_kernel<<<gblocks, gthreads, 0, st>>>(pC, Wn, bb, h.w, GV);
-      inv_kernel<<<1, 256, ism, st>>>(GV, bb, SV);
+      // the Gram matrix and its inverse do not feed the contraction: they
+      // run on the side stream while it streams R
+      cudaEventRecord(ev_fork, st);
+      cudaStreamWaitEvent(side, ev_fork, 0);
+      gram_kernel<<<gblocks, gthreads, 0, side>>>(pC, Wn, bb, h.w, GV);
+      inv_kernel<<<1, 256, 0, side>>>(GV, bb, SV);
+      cudaEventRecord(ev_join, side);
       if (tc)
-        tc_contract_rv(R, m, n, Vm, Vs, h.w, bb, klenP, splitP, Pp, st);
+        tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, klenP, splitP, Pp, st);
       else
         rv_kernel<<<dim3(tiles_m, splitP), 256, 0, st>>>(R, m, n, Vm, Vs, h.w, bb, klenP, Pp);
-      target_kernel<<<tgtU, 256, 0, st>>>(Pp, splitP, m, bb, SV, T, Cs);
-      tern_kernel<<<(Wm * 32 + 255) / 256, 256, 0, st>>>(T, m, bb, Cs, tgtU, tau, Um, Us, pB, Wm);
-      gram_kernel<<<gblocks, gthreads, 0, st>>>(pB, Wm, bb, nullptr, GU);
-      inv_kernel<<<1, 256, ism, st>>>(GU, bb, SU);
+      cudaStreamWaitEvent(st, ev_join, 0);
+      tgtP<<<tgtU, 256, kTgtSmem, st>>>(Pp, splitP, m, bb, SV, tau, T, Cs, tick, thr,
+                                                 nullptr);
+      tern_kernel<<<(Wm * 32 + 63) / 64, 64, 0, st>>>(T, m, bb, thr, Um, Us, pB, Wm, BopU);
+      cudaEventRecord(ev_fork, st);
+      cudaStreamWaitEvent(side, ev_fork, 0);
+      gram_kernel<<<gblocks, gthreads, 0, side>>>(pB, Wm, bb, nullptr, GU);
+      inv_kernel<<<1, 256, 0, side>>>(GU, bb, SU);
+      cudaEventRecord(ev_join, side);
       if (tc)
-        tc_contract_rtu(R, m, n, Um, Us, bb, klenQ, splitQ, Qp, st);
+        tc_contract_rtu(R, m, n, Um, Us, BopU, bb, klenQ, splitQ, Qp, st);
       else
         rtu_kernel<<<dim3(tiles_n, splitQ), 256, 0, st>>>(R, m, n, Um, Us, bb, klenQ, Qp);
-      target_kernel<<<tgtV, 256, 0, st>>>(Qp, splitQ, n, bb, SU, T, Cs);
-      tern_kernel<<<(Wn * 32 + 255) / 256, 256, 0, st>>>(T, n, bb, Cs, tgtV, tau, Vm, Vs, pC, Wn);
+      cudaStreamWaitEvent(st, ev_join, 0);
+      tgtQ<<<tgtV, 256, kTgtSmem, st>>>(Qp, splitQ, n, bb, SU, tau, T, Cs, tick, thr,
+                                                 it == h.iters - 1 ? Qs : nullptr);
+      tern_kernel<<<(Wn * 32 + 63) / 64, 64, 0, st>>>(T, n, bb, thr, Vm, Vs, pC, Wn, BopV);
       if (tr) {
         u64* at = tr + 2 * (size_t)n + (size_t)it * 2 * ((size_t)m + n);
         record(at, Um, Us, m);
@@ -842,15 +1223,20 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
       }
     }
     gram_kernel<<<gblocks, gthreads, 0, st>>>(pC, Wn, bb, h.w, GV);
-    rpart_kernel<<<tgtV, 256, 0, st>>>(Qp, splitQ, n, bb, Vm, Vs, h.w, Rp);
-    dsolve_kernel<<<1, 256, dsm, st>>>(GU, GV, Rp, tgtV, bb, scal, c0, h.D, h.energy, dblk);
-    deflate_kernel<<<dim3((m + 7) / 8, nch), 256, 0, st>>>(R, m, n, Um, Us, Vm, Vs, dblk, h.w, rhop);
+    rpart_kernel<<<tgtV, 256, 0, st>>>(Qs, n, bb, Vm, Vs, h.w, Rp);
+    dsolve_kernel<<<1, 256, 0, st>>>(GU, GV, Rp, tgtV, bb, scal, c0, h.D, h.energy, dblk);
+    deflate_kernel<<<dim3((m + 15) / 16, nch), 256, 0, st>>>(R, m, n, Um, Us, Vm, Vs, dblk, h.w, rhop);
     chk();
   }
   int* status = status_word_ptr();
   if (status) set_status_kernel<<<1, 1, 0, st>>>(bad, status);
   chk();
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == EXTERND_OK) rc = EXTERND_ERR_CUDA;
+  // every side-stream launch is joined into st; the handles go once the
+  // queued work no longer needs them (destruction is deferred by CUDA)
+  cudaEventDestroy(ev_fork);
+  cudaEventDestroy(ev_join);
+  cudaStreamDestroy(side);
   return rc;
 }
 

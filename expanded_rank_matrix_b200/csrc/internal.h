@@ -48,12 +48,15 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st);
 int reconstruct(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
                 int64_t k, float* out, cudaStream_t st);
 int* status_word_ptr();
+// Block-ALS contractions on the tensor cores.  Vm/Vs (Um/Us) are the 64-bit
+// per-entry masks of the ternary operand, Bop the same codes as bf16 B chunks
+// (4 KB per 32 entries); wpad the weights zero padded to a multiple of 32.
 int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
-                   const unsigned long long* Vs, const float* w, int bb, int klen, int splits,
-                   float* Pp, cudaStream_t st);
+                   const unsigned long long* Vs, const unsigned char* Bop, const float* w,
+                   const float* wpad, int bb, int klen, int splits, float* Pp, cudaStream_t st);
 int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
-                    const unsigned long long* Us, int bb, int klen, int splits, float* Qp,
-                    cudaStream_t st);
+                    const unsigned long long* Us, const unsigned char* Bop, int bb, int klen,
+                    int splits, float* Qp, cudaStream_t st);
 int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
                                cudaStream_t st);
 

@@ -18,26 +18,25 @@
 // EXTERND_ERR_TIMEOUT, the CTA stops issuing, drains (bounded) and frees its
 // tensor memory.  Outputs are split-K partials Xp[split][row][64].
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
+#include <cstdlib>
 
 #include "common.cuh"
 #include "internal.h"
+#include "umma_layout.cuh"
 
 namespace externd {
 namespace umma {
 
 typedef unsigned long long u64;
 
-constexpr int kM = 128;      // accumulator rows (TMEM lanes)
-constexpr int kN = 64;       // components (TMEM columns)
-constexpr int kKc = 32;      // K chunk
 constexpr int kThreads = 256;
 constexpr int kPartBytes = kM * kKc * 2;   // one bf16 part of the A chunk: 8 KB
-constexpr int kBBytes = kN * kKc * 2;      // B chunk: 4 KB
-constexpr int kSboK = 8 * kKc * 2;         // K-major: bytes between 8-row groups
 constexpr int kLboMN = kM / 8 * 128;       // MN-major: bytes between 8-k groups
 constexpr int kStageBytes = 3 * kPartBytes + kBBytes;
 constexpr int kSmemBytes = 2 * kStageBytes + 1024;  // 56 KB + alignment slack: 3-4 CTAs per SM
@@ -153,12 +152,6 @@ __device__ __forceinline__ uint32_t pack2(__nv_bfloat16 a, __nv_bfloat16 b) {
   return (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
 }
 
-// K-major no-swizzle offset of element (row, k) of a [rows x kKc] bf16 tile:
-// core matrices of 8 rows x 16 B; K-adjacent cores 128 B apart (LBO),
-// 8-row groups kSboK bytes apart (SBO).
-__device__ __forceinline__ uint32_t kmaj_off(int row, int k) {
-  return (uint32_t)((row >> 3) * kSboK + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
-}
 // MN-major no-swizzle offset of element (mn, k) of a [128 x kKc] bf16 tile:
 // core matrices of 8 k-rows x 16 B (8 mn); MN-adjacent cores 128 B apart (SBO),
 // K groups of 8 kLboMN bytes apart (LBO).
@@ -374,39 +367,375 @@ __global__ void __launch_bounds__(kThreads, 1) contract_kernel(
   if (wid == 0) tmem_dealloc(tmem, kN);
 }
 
+
+// ===========================================================================
+// Pipelined variant (row stride a multiple of 16 bytes).  Per K chunk the
+// producer copies into one stage of the fp32 ring: the tile of R (TMA tensor
+// copy), the chunk's ternary B operand, already laid out for the MMA (bulk
+// copy), and, for P = R W V, the chunk's 32 weights (bulk copy).  Eight
+// converter warps take a stage apart and hand it back at once: they split the
+// tile into the three bf16 parts, which go straight into tensor memory -- the
+// A operand of tcgen05.mma may live there, K-major: TMEM lane = output row,
+// one 32-bit column = two consecutive K elements -- and move B into a second,
+// MMA-side ring.  So an fp32 stage is busy only for its copy and its
+// conversion, never for the MMA.  Warp roles:
+//   warp 0      producer (one lane); allocates / frees tensor memory
+//   warp 1      MMA issuer (one lane)
+//   warps 2..9  converters; warp w serves TMEM lanes 32 (w % 4) .. + 31 and
+//               K half (w - 2) / 4 of every chunk; they also run the epilogue
+// mbarriers: full / empty guard the fp32 ring (copies landed / stage read),
+// afull / aempty the A + B stages (parts stored / tcgen05.commit after the
+// chunk's MMAs), accf the accumulator.
+// ===========================================================================
+constexpr int kS32 = 4;                                 // fp32 ring depth
+constexpr int kSA = 4;                                  // A (TMEM) + B (smem) stages
+constexpr int kTileBytes32 = kM * kKc * 4;              // 16 KB fp32 tile
+constexpr int kBOff = kTileBytes32;                     // B chunk within an fp32 stage
+constexpr int kWOff = kTileBytes32 + kBBytes;           // weights of the chunk
+constexpr int kStageBytesP = kTileBytes32 + kBBytes + 1024;  // multiple of 1024
+constexpr int kBRingOff = kS32 * kStageBytesP;          // MMA-side B ring
+constexpr int kAcolsStage = 3 * (kKc / 2);              // 48 TMEM columns per A stage
+constexpr int kTmemCols = 256;                          // accumulator 64 + 4 A stages
+constexpr int kThreadsP = 320;                          // 10 warps
+constexpr int kSmemP = kBRingOff + kSA * kBBytes + 1024;
+static_assert(kN + kSA * kAcolsStage <= kTmemCols, "tensor memory budget");
+static_assert(kStageBytesP % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+
+struct PipeBars {
+  u64 full[kS32], empty[kS32], afull[kSA], aempty[kSA], accf;
+};
+
+__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)tmap), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// D (TMEM) (+)= A (TMEM) x B (shared memory descriptor)
+__device__ __forceinline__ void umma_ts_bf16(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// Bounded wait that also gives up once another thread of the CTA has
+// recorded a timeout in *abort.
+__device__ __forceinline__ bool mbar_wait_ab(uint32_t addr, uint32_t parity,
+                                             volatile int* abort) {
+  if (mbar_test(addr, parity)) return true;
+  const long long t0 = clock64();
+  unsigned spins = 0;
+  while (!mbar_test(addr, parity)) {
+    if (((++spins) & 15u) == 0u && *abort) return false;
+    if (clock64() - t0 > kWaitBudget) {
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"((uint64_t)src), "r"(bytes), "r"(mbar)
+      : "memory");
+}
+
+// MODE 0: P = R (W V), A rows = rows of R, K = columns (tile box 32 x 128,
+//         128-byte swizzle: 16-byte group g of tile row r sits at g ^ (r % 8)).
+// MODE 1: Q^T = R^T U, A rows = columns of R, K = rows (box 128 x 32, no swizzle).
+// Bop: ternary B chunks of the K range, 4 KB per 32 K entries (umma_layout.cuh).
+// wpad: for MODE 0 the weights, zero padded to a multiple of 32 (or null).
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
+    const __grid_constant__ CUtensorMap tmap, int m, int n, const unsigned char* __restrict__ Bop,
+    const float* __restrict__ wpad, int bb, int klen, float* __restrict__ Xp,
+    int* __restrict__ status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* ring = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) PipeBars bars;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int M = MODE == 0 ? m : n, Kdim = MODE == 0 ? n : m;
+  const int i0 = blockIdx.x * kM, split = blockIdx.y;
+  const int k_begin = split * klen, k_end = min(Kdim, k_begin + klen);
+  const int nchunks = k_end > k_begin ? (k_end - k_begin + kKc - 1) / kKc : 0;
+  const bool weighted = MODE == 0 && wpad != nullptr;
+  volatile int* ab = &abort_flag;
+
+  if (wid == 0) {
+    tmem_alloc(smem_u32(&tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    for (int s = 0; s < kS32; ++s) {
+      mbar_init(smem_u32(&bars.full[s]), 1);
+      mbar_init(smem_u32(&bars.empty[s]), 8);
+    }
+    for (int s = 0; s < kSA; ++s) {
+      mbar_init(smem_u32(&bars.afull[s]), 8);
+      mbar_init(smem_u32(&bars.aempty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars.accf), 1);
+    fence_mbar_init();
+    abort_flag = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+
+  if (wid == 0) {
+    if (lane == 0) {  // ---- producer ----
+      const uint32_t tx = kTileBytes32 + kBBytes + (weighted ? kKc * 4 : 0);
+      int issued = 0;
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kS32;
+        if (c >= kS32 && !mbar_wait_ab(smem_u32(&bars.empty[s]), ((c / kS32) + 1) & 1, ab))
+          break;
+        const uint32_t fb = smem_u32(&bars.full[s]);
+        const uint32_t dst = smem_u32(ring + s * kStageBytesP);
+        const int kk = k_begin + c * kKc;
+        mbar_expect_tx(fb, tx);
+        if (MODE == 0)
+          tma_load_2d(dst, &tmap, kk, i0, fb);
+        else
+          tma_load_2d(dst, &tmap, i0, kk, fb);
+        bulk_load(dst + kBOff, Bop + (size_t)(kk / kKc) * kBBytes, kBBytes, fb);
+        if (weighted) bulk_load(dst + kWOff, wpad + kk, kKc * 4, fb);
+        ++issued;
+      }
+      // every issued copy must have landed before the CTA may exit
+      for (int c = issued > kS32 ? issued - kS32 : 0; c < issued; ++c)
+        mbar_wait(smem_u32(&bars.full[c % kS32]), (uint32_t)((c / kS32) & 1));
+    }
+  } else if (wid == 1) {
+    if (lane == 0) {  // ---- MMA issuer ----
+      const uint32_t idesc = make_idesc(0);
+      for (int c = 0; c < nchunks; ++c) {
+        const int s = c % kSA;
+        if (!mbar_wait_ab(smem_u32(&bars.afull[s]), (c / kSA) & 1, ab)) break;
+        tc_fence_after();
+        const uint32_t acol = tmem + kN + s * kAcolsStage;
+        const uint32_t bbase = smem_u32(ring + kBRingOff + s * kBBytes);
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+#pragma unroll
+          for (int ks = 0; ks < kKc / 16; ++ks)
+            umma_ts_bf16(tmem, acol + p * (kKc / 2) + ks * 8,
+                         make_desc(bbase + ks * 256, 128, kSboK), idesc,
+                         (c > 0 || p > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(smem_u32(&bars.aempty[s]));
+      }
+      // completes once every MMA issued above has finished (also after an abort)
+      umma_commit(smem_u32(&bars.accf));
+    }
+  } else {
+    // ---- converters (warps 2..9) ----
+    const int quad = wid & 3;          // TMEM lanes this warp may access
+    const int kh = (wid - 2) >> 2;     // K half of each chunk
+    const int row = quad * 32 + lane;  // tile row = TMEM lane
+    const int ctid = tid - 64;         // 0..255: one 16-byte piece of B
+    for (int c = 0; c < nchunks; ++c) {
+      const int s = c % kS32, sa = c % kSA;
+      bool ok = mbar_wait_ab(smem_u32(&bars.full[s]), (c / kS32) & 1, ab);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const unsigned char* st = ring + s * kStageBytesP;
+      float x[16];
+      if (MODE == 0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int g = (kh * 4 + q) ^ (row & 7);
+          const float4 v = *(const float4*)(st + row * 128 + g * 16);
+          x[4 * q] = v.x;
+          x[4 * q + 1] = v.y;
+          x[4 * q + 2] = v.z;
+          x[4 * q + 3] = v.w;
+        }
+        if (weighted) {
+          const float* ws = (const float*)(st + kWOff) + kh * 16;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) x[e] *= ws[e];
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[e] = *(const float*)(st + (kh * 16 + e) * 512 + row * 4);
+      }
+      const uint4 bpiece = *(const uint4*)(st + kBOff + ctid * 16);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.empty[s]));  // the fp32 stage is free again
+      uint32_t ph[8], pm[8], pl[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        __nv_bfloat16 h0, m0, l0, h1, m1, l1;
+        split3(x[2 * e], h0, m0, l0);
+        split3(x[2 * e + 1], h1, m1, l1);
+        ph[e] = pack2(h0, h1);
+        pm[e] = pack2(m0, m1);
+        pl[e] = pack2(l0, l1);
+      }
+      // A / B stage sa: the MMAs of chunk c - kSA must be done with it
+      ok = c < kSA || mbar_wait_ab(smem_u32(&bars.aempty[sa]), ((c / kSA) + 1) & 1, ab);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + kN + sa * kAcolsStage + kh * 8;
+      tmem_st8(ta, ph);
+      tmem_st8(ta + kKc / 2, pm);
+      tmem_st8(ta + kKc, pl);
+      *(uint4*)(ring + kBRingOff + sa * kBBytes + ctid * 16) = bpiece;
+      tmem_st_wait();
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.afull[sa]));
+    }
+    // ---- epilogue: accumulator columns 32 kh .. 32 kh + 31 of lane `row` ----
+    mbar_wait(smem_u32(&bars.accf), 0u);
+    tc_fence_after();
+    const int gi = i0 + row;
+    float* out = Xp + ((size_t)split * M + gi) * bb;
+    if (nchunks == 0) {
+      if (gi < M)
+        for (int t = 0; t < 32; ++t)
+          if (kh * 32 + t < bb) out[kh * 32 + t] = 0.f;
+    } else if (!*ab) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[16];
+        const int col = kh * 32 + h * 16;
+        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)col, v);
+        if (gi < M)
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            if (col + t < bb) out[col + t] = __uint_as_float(v[t]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (wid == 0) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (tid == 0 && abort_flag) atomicCAS(status, 0, EXTERND_ERR_TIMEOUT);
+}
+
 }  // namespace umma
 
-// Host launchers; klen must be a multiple of kKc (32).
-int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
-                   const unsigned long long* Vs, const float* w, int bb, int klen, int splits,
-                   float* Pp, cudaStream_t st) {
+namespace {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library); resolved once.
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+// Tensor map over the row-major m x n fp32 residual: MODE 0 boxes of 128
+// rows x 32 columns (128-byte swizzle), MODE 1 boxes of 32 rows x 128 columns.
+// Out-of-range box elements read as zero.
+bool make_tmap(CUtensorMap* tm, const float* R, int m, int n, int mode) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)m};
+  const cuuint64_t strides[1] = {(cuuint64_t)n * sizeof(float)};
+  const cuuint32_t box0[2] = {(cuuint32_t)umma::kKc, (cuuint32_t)umma::kM};
+  const cuuint32_t box1[2] = {(cuuint32_t)umma::kM, (cuuint32_t)umma::kKc};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, (void*)R, dims, strides,
+            mode == 0 ? box0 : box1, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            mode == 0 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tma_ok(const float* R, int n) {
+  return (n % 4) == 0 && (((uintptr_t)R) & 15) == 0 && getenv("EXTERND_CONTRACT_NO_TMA") == nullptr;
+}
+
+void set_attrs() {
   using namespace umma;
   static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(contract_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    cudaFuncSetAttribute(contract_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    attr = true;
-  }
+  if (attr) return;
+  attr = true;
+  cudaFuncSetAttribute(contract_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(contract_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(contract_tma_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemP);
+  cudaFuncSetAttribute(contract_tma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemP);
+}
+
+}  // namespace
+
+// Host launchers; klen must be a multiple of kKc (32).  Rows of R that start
+// 16-byte aligned take the TMA-pipelined kernel, others the direct-load one.
+int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
+                   const unsigned long long* Vs, const unsigned char* Bop, const float* w,
+                   const float* wpad, int bb, int klen, int splits, float* Pp, cudaStream_t st) {
+  using namespace umma;
+  set_attrs();
   int* status = status_word_ptr();
   dim3 grid((unsigned)((m + kM - 1) / kM), (unsigned)splits);
-  contract_kernel<0><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Vm, Vs, w, bb, klen, Pp, status);
+  CUtensorMap tm;
+  if (tma_ok(R, n) && make_tmap(&tm, R, m, n, 0))
+    contract_tma_kernel<0><<<grid, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, w ? wpad : nullptr,
+                                                            bb, klen, Pp, status);
+  else
+    contract_kernel<0><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Vm, Vs, w, bb, klen, Pp,
+                                                                 status);
   return cudaGetLastError() == cudaSuccess ? EXTERND_OK : EXTERND_ERR_CUDA;
 }
 
 int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
-                    const unsigned long long* Us, int bb, int klen, int splits, float* Qp,
-                    cudaStream_t st) {
+                    const unsigned long long* Us, const unsigned char* Bop, int bb, int klen,
+                    int splits, float* Qp, cudaStream_t st) {
   using namespace umma;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(contract_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    cudaFuncSetAttribute(contract_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    attr = true;
-  }
+  set_attrs();
   int* status = status_word_ptr();
   dim3 grid((unsigned)((n + kM - 1) / kM), (unsigned)splits);
-  contract_kernel<1><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Um, Us, nullptr, bb, klen, Qp,
-                                                        status);
+  CUtensorMap tm;
+  if (tma_ok(R, n) && make_tmap(&tm, R, m, n, 1))
+    contract_tma_kernel<1><<<grid, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, nullptr, bb, klen, Qp,
+                                                            status);
+  else
+    contract_kernel<1><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Um, Us, nullptr, bb,
+                                                                 klen, Qp, status);
   return cudaGetLastError() == cudaSuccess ? EXTERND_OK : EXTERND_ERR_CUDA;
 }
 
