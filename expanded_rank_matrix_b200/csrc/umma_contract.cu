@@ -387,7 +387,12 @@ __global__ void __launch_bounds__(kThreads, 1) contract_kernel(
 // afull / aempty the A + B stages (parts stored / tcgen05.commit after the
 // chunk's MMAs), accf the accumulator.
 // ===========================================================================
-constexpr int kS32 = 4;                                 // fp32 ring depth
+// One CTA per SM: with two co-resident CTAs the transposed contraction
+// (Q^T = R^T U) returned wrong partial sums from the CTA placed second on an
+// SM (reproducible with 160-280 CTAs, varying from run to run; the same
+// grid at one CTA per SM, and the other contraction at two, were exact).
+// The shared memory a second CTA would have used deepens the fp32 ring.
+constexpr int kS32 = 8;                                 // fp32 ring depth
 constexpr int kSA = 4;                                  // A (TMEM) + B (smem) stages
 constexpr int kTileBytes32 = kM * kKc * 4;              // 16 KB fp32 tile
 constexpr int kBOff = kTileBytes32;                     // B chunk within an fp32 stage
@@ -400,6 +405,8 @@ constexpr int kThreadsP = 320;                          // 10 warps
 constexpr int kSmemP = kBRingOff + kSA * kBBytes + 1024;
 static_assert(kN + kSA * kAcolsStage <= kTmemCols, "tensor memory budget");
 static_assert(kStageBytesP % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(2 * (kSmemP + 1024) > 228 * 1024, "the ring must keep the kernel at one CTA per SM");
+static_assert(kSmemP <= 227 * 1024, "shared memory per CTA");
 
 struct PipeBars {
   u64 full[kS32], empty[kS32], afull[kSA], aempty[kSA], accf;
