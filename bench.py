@@ -6,6 +6,13 @@ projection-shaped matrix at mu = 3 (k = 7680 components, tau = 0.5, 6 ALS
 iterations, block = 1) through the C ABI.  Prints one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload attn2560|mlp9728_b64|mlp9728_b1|block_layer]
+  python bench.py --case attn2560_k64|mlp9728_3blocks     (small profiling cases)
+
+--workload picks another configuration (default: the 2560 x 2560 one above);
+mlp9728_b64 / _b1 decompose the 9728 x 2560 MLP-shaped matrix (mu = 2) with
+block-ALS (b = 64) or the sequential kernel, block_layer the seven importance-
+weighted matrices of one transformer block (mu = 3, b = 64) per step.
 
 --impl reference times the CPU oracle (oracle/externd_ref.cpp, single
 thread) on a bounded prefix of the same workload.  With N > 1 (torchrun)
@@ -39,9 +46,47 @@ def _env_int(name, default):
         return default
 
 
-def _workload():
+WORKLOADS = ("attn2560", "mlp9728_b64", "mlp9728_b1", "block_layer")
+
+
+def _workloads(name="attn2560"):
+    """The matrices one step decomposes."""
     from expanded_rank_matrix_b200 import workloads as W
-    return W.config_attn2560()
+    if name == "attn2560":
+        return [W.config_attn2560()]
+    if name == "mlp9728_b64":
+        return [W.config_mlp9728(64)]
+    if name == "mlp9728_b1":
+        return [W.config_mlp9728(1)]
+    if name == "block_layer":
+        return W.config_block_matrices(64)
+    raise SystemExit(f"unknown workload {name}")
+
+
+def _workload():
+    return _workloads()[0]
+
+
+def _launches_per_decomposition(wl):
+    """Kernels this library launches for one decomposition of wl (block path:
+    the fixed per-block sequence of block_als.cu)."""
+    if wl.block <= 1:
+        return 1
+    nb = (wl.k + wl.block - 1) // wl.block
+    per_block = 3 + wl.iters * 10 + 4  # select, vinit, planes; 2 x (gram, inv, contract, target, tern); gram, rpart, dsolve, deflate
+    return 1 + (1 if wl.w is not None else 0) + nb * per_block + 1  # setup (+ weight check) ... status
+
+
+def max_over_ranks(seconds: float, world: int, device=None) -> float:
+    """The slowest rank's time: every rank contributes its own device time and
+    all of them get the maximum (a collective when world > 1)."""
+    if world <= 1:
+        return seconds
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def _config(wl, extra=None):
@@ -150,8 +195,8 @@ def _oracle_prefix(wl, ncomp: int):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl = _workload()
-    ncomp = _env_int("EXTERND_REF_COMPONENTS", 24)
+    wl = _workloads(args.workload)[0]
+    ncomp = _env_int("EXTERND_REF_COMPONENTS", 24 if wl.block <= 1 else wl.block)
     for _ in range(args.warmup):
         _oracle_prefix(wl, ncomp)
     times = [_oracle_prefix(wl, ncomp) for _ in range(args.steps)]
@@ -175,23 +220,23 @@ def run_reference(args, rank, world):
 # CUDA path
 # ---------------------------------------------------------------------------
 def run_ours(args, rank, world, local_rank):
-    import numpy as np
     import torch
-    import torch.distributed as dist
 
     from expanded_rank_matrix_b200 import externd as X
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = _workload()
-    m, n, k = wl.m, wl.n, wl.k
-    A = torch.from_numpy(wl.a).to(dev)
-    out = X.alloc_factors(m, n, k, dev)
+    wls = _workloads(args.workload)
+    As = [torch.from_numpy(wl.a).to(dev) for wl in wls]
+    Ws = [None if wl.w is None else torch.from_numpy(wl.w).to(dev) for wl in wls]
+    outs = [X.alloc_factors(wl.m, wl.n, wl.k, dev) for wl in wls]
+    k_step = sum(wl.k for wl in wls)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def step():
-        X.decompose_into(out, A, wl.mu, wl.tau, wl.iters, stream=stream)
+    def step(srcs=As):
+        for wl, A, w, out in zip(wls, srcs, Ws, outs):
+            X.decompose_into(out, A, wl.mu, wl.tau, wl.iters, w=w, block=wl.block, stream=stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -202,6 +247,7 @@ def run_ours(args, rank, world, local_rank):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
@@ -217,20 +263,17 @@ def run_ours(args, rank, world, local_rank):
     if status != X.OK:
         raise SystemExit(f"device status {status} in the timed region")
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    tot_ms = torch.tensor([sum(step_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tot_ms, op=dist.ReduceOp.MAX)
-    tot_s = float(tot_ms.item()) / 1000.0
-    value = world * k * args.steps / tot_s
-    energy = float(out.energy[-1].item())
+    tot_s = max_over_ranks(sum(step_ms) / 1000.0, world, dev)
+    value = world * k_step * args.steps / tot_s
+    energies = [float(out.energy[-1].item()) for out in outs]
 
     # end to end through host buffers: pinned A in, packed factors out
-    hA = torch.from_numpy(wl.a).pin_memory()
-    hB = torch.empty(out.packed_B.shape, dtype=torch.int32).pin_memory()
-    hC = torch.empty(out.packed_C.shape, dtype=torch.int32).pin_memory()
-    hD = torch.empty(k, dtype=torch.float32).pin_memory()
-    hE = torch.empty(k, dtype=torch.float64).pin_memory()
-    A2 = torch.empty_like(A)
+    hAs = [torch.from_numpy(wl.a).pin_memory() for wl in wls]
+    hout = [(torch.empty(o.packed_B.shape, dtype=torch.int32).pin_memory(),
+             torch.empty(o.packed_C.shape, dtype=torch.int32).pin_memory(),
+             torch.empty(o.D.shape, dtype=torch.float32).pin_memory(),
+             torch.empty(o.energy.shape, dtype=torch.float64).pin_memory()) for o in outs]
+    A2s = [torch.empty_like(A) for A in As]
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:
@@ -239,63 +282,105 @@ def run_ours(args, rank, world, local_rank):
     for s in range(args.steps):
         flush.zero_()
         e2e_ev[s][0].record(stream)
-        A2.copy_(hA, non_blocking=True)
-        X.decompose_into(out, A2, wl.mu, wl.tau, wl.iters, stream=stream)
-        hB.copy_(out.packed_B, non_blocking=True)
-        hC.copy_(out.packed_C, non_blocking=True)
-        hD.copy_(out.D, non_blocking=True)
-        hE.copy_(out.energy, non_blocking=True)
+        for A2, hA in zip(A2s, hAs):
+            A2.copy_(hA, non_blocking=True)
+        step(A2s)
+        for o, (hB, hC, hD, hE) in zip(outs, hout):
+            hB.copy_(o.packed_B, non_blocking=True)
+            hC.copy_(o.packed_C, non_blocking=True)
+            hD.copy_(o.D, non_blocking=True)
+            hE.copy_(o.energy, non_blocking=True)
         e2e_ev[s][1].record(stream)
     torch.cuda.synchronize()
     if X.sync_status(stream) != X.OK:
         raise SystemExit("device status error in the end-to-end leg")
-    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in e2e_ev)], dtype=torch.float64,
-                          device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * k * args.steps / (float(e2e_ms.item()) / 1000.0)
-    h2d = hA.numel() * 4
-    d2h = hB.numel() * 4 + hC.numel() * 4 + hD.numel() * 4 + hE.numel() * 8
-    if abs(float(hE[-1]) - energy) > 1e-12:
-        raise SystemExit("end-to-end result differs from the device-timed result")
+    e2e_s = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1000.0, world, dev)
+    e2e_value = world * k_step * args.steps / e2e_s
+    h2d = sum(hA.numel() * 4 for hA in hAs)
+    d2h = sum(hB.numel() * 4 + hC.numel() * 4 + hD.numel() * 4 + hE.numel() * 8
+              for hB, hC, hD, hE in hout)
+    for (_, _, _, hE), e in zip(hout, energies):
+        if abs(float(hE[-1]) - e) > 1e-12:
+            raise SystemExit("end-to-end result differs from the device-timed result")
 
     if rank != 0:
         return
-    # roofline of the dominant (only) kernel of the step
-    per_comp = 4.0 * m * n * (2 * wl.iters + 2)
-    alg_bytes = per_comp * k
-    avg_s = tot_s / args.steps if world == 1 else (sum(step_ms) / 1000.0) / args.steps
+    # roofline: algorithmic residual traffic, 4 m n (2I + 2) bytes per component
+    # (sequential) or per block of components (block-ALS)
+    alg_bytes = 0.0
+    for wl in wls:
+        units = wl.k if wl.block <= 1 else (wl.k + wl.block - 1) // wl.block
+        alg_bytes += 4.0 * wl.m * wl.n * (2 * wl.iters + 2) * units
+    avg_s = (sum(step_ms) / 1000.0) / args.steps
     achieved = alg_bytes / avg_s / 1e9
     peak, peak_kind = _peaks()
-    traffic = _profiled_traffic("seq_als_kernel", wl.name)
+    sequential = all(wl.block <= 1 for wl in wls)
+    kernel = "seq_als_kernel" if sequential else "block-ALS path (all kernels of the step)"
+    traffic = _profiled_traffic(kernel, wls[0].name) if len(wls) == 1 else None
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-            "kernel": "seq_als_kernel",
-            "alg_bytes_per_launch": alg_bytes,
-            "note": "residual R is resident in shared memory across the grid; algorithmic "
-                    "bytes = 4*m*n*(2I+2) per component"}
+            "kernel": kernel, "alg_bytes_per_launch": alg_bytes if sequential else None,
+            "alg_bytes_per_step": alg_bytes,
+            "note": ("residual R is resident in shared memory across the grid; algorithmic "
+                     "bytes = 4*m*n*(2I+2) per component" if sequential else
+                     "algorithmic bytes = 4*m*n*(2I+2) per block of b components (2I "
+                     "contractions + deflation read/write); achieved over the whole step")}
+    if len(wls) == 1:
+        cfg = _config(wls[0])
+    else:
+        cfg = {"workload": f"{args.workload}: " + ", ".join(f"{wl.name} {wl.m}x{wl.n}" for wl in wls)
+               + f"; mu={wls[0].mu:g}, tau={wls[0].tau:g}, I={wls[0].iters}, block={wls[0].block}, "
+               "importance-weighted", "k_total": k_step,
+               "matrices": [{"name": wl.name, "m": wl.m, "n": wl.n, "k": wl.k} for wl in wls]}
+    cfg.update({"parallelism": f"replicas x{world}",
+                "l2": "flushed between timed steps (256 MiB write outside the per-step events)",
+                "achieved_gbs": achieved})
+    if len(wls) == 1:
+        cfg["energy_preserved_pct"] = 100.0 * energies[0]
+    else:
+        cfg["energy_preserved_pct"] = {wl.name: 100.0 * e for wl, e in zip(wls, energies)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sum(step_ms) / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": _config(wl, {"parallelism": f"replicas x{world}",
-                                   "l2": "flushed between timed steps (256 MiB write outside "
-                                         "the per-step events)",
-                                   "achieved_gbs": achieved,
-                                   "energy_preserved_pct": 100.0 * energy}),
-            "roofline": roof,
+            "config": cfg, "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * sum(_launches_per_decomposition(wl) for wl in wls),
             "clocks": clk.summary(),
             "step_ms": step_ms}
     if world == 1 and not args.no_cpu_baseline:
-        ncomp = _env_int("EXTERND_CPU_COMPONENTS", 96)
-        t = _oracle_prefix(wl, ncomp)
+        wl0 = wls[0]
+        ncomp = _env_int("EXTERND_CPU_COMPONENTS", 96 if wl0.block <= 1 else 2 * wl0.block)
+        t = _oracle_prefix(wl0, ncomp)
         line["cpu_baseline"] = {"value": ncomp / t, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": f"first {ncomp} of {k} components, free-running "
-                                          f"oracle from A, one thread"}
+                                "sample": f"first {ncomp} of {wl0.k} components of {wl0.name}, "
+                                          f"free-running oracle from A, one thread"}
     print(json.dumps(line), flush=True)
+
+
+def run_case(args):
+    """Small cases for ncu captures: the same calls, twice, no timing."""
+    import torch
+
+    from expanded_rank_matrix_b200 import externd as X
+    from expanded_rank_matrix_b200 import workloads as W
+    if args.case == "attn2560_k64":
+        wl = W.config_attn2560()
+        mu, block = 64 / min(wl.m, wl.n), 1
+    elif args.case == "mlp9728_3blocks":
+        wl = W.config_mlp9728(64)
+        mu, block = 3 * 64 / min(wl.m, wl.n), 64
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    A = torch.from_numpy(wl.a).cuda()
+    for _ in range(2):
+        f = X.decompose(A, mu, wl.tau, wl.iters, block=block)
+    torch.cuda.synchronize()
+    st = X.sync_status()
+    print(json.dumps({"case": args.case, "k": f.k, "energy": float(f.energy[-1]), "status": st}))
+    if st != X.OK:
+        raise SystemExit(1)
 
 
 def main():
@@ -305,7 +390,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=WORKLOADS, default="attn2560")
+    ap.add_argument("--case", choices=("attn2560_k64", "mlp9728_3blocks"), default=None)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     rank = _env_int("RANK", 0)
