@@ -582,8 +582,11 @@ __global__ void __launch_bounds__(256) rtu_kernel(const float* __restrict__ R, i
 // thr[l] = tau * rms(T[:, l]), then rearms the counter.  With Xout set, the
 // split-summed X (rows x bb, fp64) is stored as well.
 constexpr int kTgtRows2 = 64;  // rows per CTA of target_kernel
-constexpr int kMaxSplits = 16; // split-K partials per contraction
+constexpr int kMaxSplits = kMaxSegs;  // partials per output row (split-K or stream-K)
 constexpr int kXs = kTgtRows2 + 2;  // padded row of the transposed tile (16-byte aligned)
+// Partials: split-K layout Xp[split][row][bb] (sk == 0, `splits` of them) or
+// stream-K layout Xp[(t Sslots + slot) 128 + row % 128][bb] with the tile's
+// segment count from the plan (C, U, G) (sk != 0).
 template <int NS>
 __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict__ Xp, int splits,
                                                         int rows, int bb,
@@ -592,7 +595,8 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
                                                         double* __restrict__ colss,
                                                         unsigned* __restrict__ ticket,
                                                         double* __restrict__ thr,
-                                                        double* __restrict__ Xout) {
+                                                        double* __restrict__ Xout, int sk, int C,
+                                                        long long U, int G, int Sslots) {
   extern __shared__ __align__(16) double tsh[];
   double* Ss = tsh;                                                 // [64][64]: S[l2][l]
   double* Xt = tsh + kMaxB * kMaxB;                                 // [64][kXs]
@@ -613,7 +617,9 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
   {
     // thread: columns lq .. lq+3 (lq = 4 (tid % 16)), rows tid / 16 + 16 h
     const int lq = (tid & 15) * 4, rr = tid >> 4;
-    const size_t sstride = (size_t)rows * bb;
+    // 64-row CTAs never straddle a 128-row tile
+    const int nparts = sk ? umma::sk_nseg(x0 / umma::kM, C, U, G) : splits;
+    const size_t sstride = sk ? (size_t)umma::kM * bb : (size_t)rows * bb;
     const bool vec = (bb & 3) == 0;
     constexpr int RPR = NS > 8 ? 1 : 2;  // rows per round: at most 64 floats in flight
 #pragma unroll 1
@@ -623,11 +629,14 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
       for (int h = 0; h < RPR; ++h) {
         const int x = x0 + rr + 16 * (h0 + h);
         const bool ok = x < rows && lq < bb;
-        const float* src = Xp + (size_t)(ok ? x : 0) * bb + (ok ? lq : 0);
+        const int xs = ok ? x : 0;
+        const size_t prow = sk ? ((size_t)(xs / umma::kM) * Sslots * umma::kM + xs % umma::kM)
+                               : (size_t)xs;
+        const float* src = Xp + prow * bb + (ok ? lq : 0);
 #pragma unroll
         for (int sp = 0; sp < NS; ++sp) {
           float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (ok && sp < splits) {
+          if (ok && sp < nparts) {
             const float* q = src + sp * sstride;
             if (vec) {
               t = __ldg((const float4*)q);
@@ -646,7 +655,7 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
         double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
 #pragma unroll
         for (int sp = 0; sp < NS; ++sp)
-          if (sp < splits) {
+          if (sp < nparts) {
             s0 += (double)v[h][sp].x;
             s1 += (double)v[h][sp].y;
             s2 += (double)v[h][sp].z;
@@ -748,7 +757,7 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
 constexpr size_t kTgtSmem = sizeof(double) * (kMaxB * kMaxB + kMaxB * kXs + 16 * kMaxB);
 // the target kernel instantiated for a split-count bound
 typedef void (*TargetFn)(const float*, int, int, int, const double*, double, double*, double*,
-                         unsigned*, double*, double*);
+                         unsigned*, double*, double*, int, int, long long, int, int);
 inline TargetFn target_for(int splits) {
   if (splits <= 1) return target_kernel<1>;
   if (splits <= 2) return target_kernel<2>;
@@ -1069,6 +1078,17 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
   const int klenQ = ((m + splitQ - 1) / splitQ + kq - 1) / kq * kq;
   splitP = (n + klenP - 1) / klenP;
   splitQ = (m + klenQ - 1) / klenQ;
+  // the persistent TMA contraction (stream-K partials) whenever R's rows are
+  // TMA-addressable; the workspace keeps R at a 256-byte aligned offset
+  const bool sk = tc && tc_contract_tma_ok(n);
+  TcPlan planP{}, planQ{};
+  if (sk) {
+    tc_contract_plan(m, n, nsm, &planP);
+    tc_contract_plan(n, m, nsm, &planQ);
+  }
+  const size_t partsP = sk ? (size_t)planP.T * planP.S * 128 : (size_t)splitP * m;
+  const size_t partsQ = sk ? (size_t)planQ.T * planQ.S * 128 : (size_t)splitQ * n;
+  const int boundP = sk ? planP.S : splitP, boundQ = sk ? planQ.S : splitQ;
   const int tgtU = (m + kTgtRows2 - 1) / kTgtRows2, tgtV = (n + kTgtRows2 - 1) / kTgtRows2;
   const int nch = (n + kChunk - 1) / kChunk;
   const int mx = std::max(m, n);
@@ -1086,8 +1106,8 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
   const size_t oRows = take(sizeof(int) * kMaxB);
   const size_t oUm = take(sizeof(u64) * m), oUs = take(sizeof(u64) * m);
   const size_t oVm = take(sizeof(u64) * n), oVs = take(sizeof(u64) * n);
-  const size_t oPp = take(sizeof(float) * (size_t)splitP * m * b);
-  const size_t oQp = take(sizeof(float) * (size_t)splitQ * n * b);
+  const size_t oPp = take(sizeof(float) * partsP * b);
+  const size_t oQp = take(sizeof(float) * partsQ * b);
   const size_t oT = take(sizeof(double) * (size_t)mx * b);
   const size_t oCs = take(sizeof(double) * (size_t)std::max(tgtU, tgtV) * b);
   const size_t oRp = take(sizeof(double) * (size_t)tgtV * b);
@@ -1142,7 +1162,7 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
     cudaFreeAsync(ws, st);
     return EXTERND_ERR_CUDA;
   }
-  const TargetFn tgtP = target_for(splitP), tgtQ = target_for(splitQ);
+  const TargetFn tgtP = target_for(boundP), tgtQ = target_for(boundQ);
   cudaFuncSetAttribute(tgtP, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgtSmem);
   cudaFuncSetAttribute(tgtQ, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgtSmem);
   // the row-energy keys of the radix select stay in shared memory when they fit
@@ -1196,12 +1216,13 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
       inv_kernel<<<1, 256, 0, side>>>(GV, bb, SV);
       cudaEventRecord(ev_join, side);
       if (tc)
-        tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, klenP, splitP, Pp, st);
+        tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, sk ? &planP : nullptr, klenP, splitP,
+                       Pp, st);
       else
         rv_kernel<<<dim3(tiles_m, splitP), 256, 0, st>>>(R, m, n, Vm, Vs, h.w, bb, klenP, Pp);
       cudaStreamWaitEvent(st, ev_join, 0);
-      tgtP<<<tgtU, 256, kTgtSmem, st>>>(Pp, splitP, m, bb, SV, tau, T, Cs, tick, thr,
-                                                 nullptr);
+      tgtP<<<tgtU, 256, kTgtSmem, st>>>(Pp, splitP, m, bb, SV, tau, T, Cs, tick, thr, nullptr, sk,
+                                         planP.C, planP.U, planP.G, planP.S);
       tern_kernel<<<(Wm * 32 + 63) / 64, 64, 0, st>>>(T, m, bb, thr, Um, Us, pB, Wm, BopU);
       cudaEventRecord(ev_fork, st);
       cudaStreamWaitEvent(side, ev_fork, 0);
@@ -1209,12 +1230,13 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
       inv_kernel<<<1, 256, 0, side>>>(GU, bb, SU);
       cudaEventRecord(ev_join, side);
       if (tc)
-        tc_contract_rtu(R, m, n, Um, Us, BopU, bb, klenQ, splitQ, Qp, st);
+        tc_contract_rtu(R, m, n, Um, Us, BopU, bb, sk ? &planQ : nullptr, klenQ, splitQ, Qp, st);
       else
         rtu_kernel<<<dim3(tiles_n, splitQ), 256, 0, st>>>(R, m, n, Um, Us, bb, klenQ, Qp);
       cudaStreamWaitEvent(st, ev_join, 0);
       tgtQ<<<tgtV, 256, kTgtSmem, st>>>(Qp, splitQ, n, bb, SU, tau, T, Cs, tick, thr,
-                                                 it == h.iters - 1 ? Qs : nullptr);
+                                         it == h.iters - 1 ? Qs : nullptr, sk, planQ.C, planQ.U,
+                                         planQ.G, planQ.S);
       tern_kernel<<<(Wn * 32 + 63) / 64, 64, 0, st>>>(T, n, bb, thr, Vm, Vs, pC, Wn, BopV);
       if (tr) {
         u64* at = tr + 2 * (size_t)n + (size_t)it * 2 * ((size_t)m + n);

@@ -51,12 +51,23 @@ int* status_word_ptr();
 // Block-ALS contractions on the tensor cores.  Vm/Vs (Um/Us) are the 64-bit
 // per-entry masks of the ternary operand, Bop the same codes as bf16 B chunks
 // (4 KB per 32 entries); wpad the weights zero padded to a multiple of 32.
+// With a plan (and 16-byte aligned rows of R) the persistent TMA kernel runs
+// and writes stream-K tile partials Xp[(t S + slot) 128 + row][bb]; otherwise
+// the direct kernel writes split-K partials Xp[split][row][bb].
+constexpr int kMaxSegs = 16;  // partials summed per output row, either layout
+struct TcPlan {
+  int T, C, G, S;  // tiles of 128 rows, chunks of 32 along K, CTAs, slots per tile
+  long long U;     // T * C units
+};
+void tc_contract_plan(int M, int Kdim, int nsm, TcPlan* p);
+bool tc_contract_tma_ok(int n);  // n % 4 == 0 and the tensor-map encoder is available
 int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
                    const unsigned long long* Vs, const unsigned char* Bop, const float* w,
-                   const float* wpad, int bb, int klen, int splits, float* Pp, cudaStream_t st);
+                   const float* wpad, int bb, const TcPlan* p, int klen, int splits, float* Pp,
+                   cudaStream_t st);
 int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
-                    const unsigned long long* Us, const unsigned char* Bop, int bb, int klen,
-                    int splits, float* Qp, cudaStream_t st);
+                    const unsigned long long* Us, const unsigned char* Bop, int bb, const TcPlan* p,
+                    int klen, int splits, float* Qp, cudaStream_t st);
 int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
                                cudaStream_t st);
 

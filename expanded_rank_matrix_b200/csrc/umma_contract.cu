@@ -23,6 +23,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstdlib>
 
@@ -369,47 +370,55 @@ __global__ void __launch_bounds__(kThreads, 1) contract_kernel(
 
 
 // ===========================================================================
-// Pipelined variant (row stride a multiple of 16 bytes).  Per K chunk the
-// producer copies into one stage of the fp32 ring: the tile of R (TMA tensor
-// copy), the chunk's ternary B operand, already laid out for the MMA (bulk
-// copy), and, for P = R W V, the chunk's 32 weights (bulk copy).  Eight
-// converter warps take a stage apart and hand it back at once: they split the
-// tile into the three bf16 parts, which go straight into tensor memory -- the
-// A operand of tcgen05.mma may live there, K-major: TMEM lane = output row,
-// one 32-bit column = two consecutive K elements -- and move B into a second,
-// MMA-side ring.  So an fp32 stage is busy only for its copy and its
-// conversion, never for the MMA.  Warp roles:
-//   warp 0      producer (one lane); allocates / frees tensor memory
-//   warp 1      MMA issuer (one lane)
-//   warps 2..9  converters; warp w serves TMEM lanes 32 (w % 4) .. + 31 and
-//               K half (w - 2) / 4 of every chunk; they also run the epilogue
-// mbarriers: full / empty guard the fp32 ring (copies landed / stage read),
-// afull / aempty the A + B stages (parts stored / tcgen05.commit after the
-// chunk's MMAs), accf the accumulator.
-// ===========================================================================
+// Pipelined, persistent variant (row stride a multiple of 16 bytes): one CTA
+// per SM, each taking an equal contiguous run of the (tile, K-chunk) units of
+// the contraction (stream-K partition, umma_layout.cuh), so every SM streams
+// R for the whole launch.  Per chunk the producer copies into one stage of
+// the fp32 ring: the 128 x 32 tile of R (TMA tensor copy), the chunk's
+// ternary B operand, already laid out for the MMA (bulk copy), and, for
+// P = R W V, the chunk's 32 weights (bulk copy).  Converter warps split the
+// tile into the three bf16 parts, which go straight into the stage's slice of
+// tensor memory -- the A operand of tcgen05.mma may live there, K-major:
+// TMEM lane = output row, one 32-bit column = two consecutive K elements;
+// B is read by the MMA where the copy put it.  A stage (tile, B and A slice)
+// is handed back to the producer by the tcgen05.commit after its MMAs.  Two
+// accumulators in tensor memory alternate between the CTA's tile
+// segments, so a finished segment is read out while the next one streams.
+// Warp roles:
+//   warp 0        producer (one lane); allocates / frees tensor memory
+//   warp 1        MMA issuer (one lane)
+//   warps 2..5    epilogue: accumulator -> split-K partial of the segment
+//   warps 6..21   converters, two groups of eight on alternate chunks; warp w
+//                 serves TMEM lanes 32 (w % 4) .. + 31 and K half
+//                 ((w - 6) / 4) % 2 of its group's chunks
+// mbarriers per stage: full (copies landed), afull (A parts stored), aempty
+// (tcgen05.commit after the chunk's MMAs); accf / accfree the two
+// accumulators (segment's MMAs done / read out); drain the final commit.
 // One CTA per SM: with two co-resident CTAs the transposed contraction
 // (Q^T = R^T U) returned wrong partial sums from the CTA placed second on an
-// SM (reproducible with 160-280 CTAs, varying from run to run; the same
-// grid at one CTA per SM, and the other contraction at two, were exact).
-// The shared memory a second CTA would have used deepens the fp32 ring.
-constexpr int kS32 = 8;                                 // fp32 ring depth
-constexpr int kSA = 4;                                  // A (TMEM) + B (smem) stages
+// SM (reproducible with 160-280 CTAs, varying from run to run; one CTA per
+// SM was exact); the shared memory a second CTA would use deepens the ring.
+// ===========================================================================
+constexpr int kS32 = 8;                                 // ring depth (fp32 tile + B + A stage)
 constexpr int kTileBytes32 = kM * kKc * 4;              // 16 KB fp32 tile
-constexpr int kBOff = kTileBytes32;                     // B chunk within an fp32 stage
+constexpr int kBOff = kTileBytes32;                     // B chunk within a stage
 constexpr int kWOff = kTileBytes32 + kBBytes;           // weights of the chunk
 constexpr int kStageBytesP = kTileBytes32 + kBBytes + 1024;  // multiple of 1024
-constexpr int kBRingOff = kS32 * kStageBytesP;          // MMA-side B ring
 constexpr int kAcolsStage = 3 * (kKc / 2);              // 48 TMEM columns per A stage
-constexpr int kTmemCols = 256;                          // accumulator 64 + 4 A stages
-constexpr int kThreadsP = 320;                          // 10 warps
-constexpr int kSmemP = kBRingOff + kSA * kBBytes + 1024;
-static_assert(kN + kSA * kAcolsStage <= kTmemCols, "tensor memory budget");
+constexpr int kAcc0 = 0, kAstage0 = 2 * kN;             // TMEM: 2 accumulators, then A stages
+constexpr int kTmemCols = 512;
+constexpr int kEpiWarps = 4;
+constexpr int kConvWarp0 = 2 + kEpiWarps;
+constexpr int kConvGroups = 2;                          // converter groups, alternate chunks
+constexpr int kThreadsP = 32 * kConvWarp0 + 256 * kConvGroups;
+constexpr int kSmemP = kS32 * kStageBytesP + 1024;
+static_assert(kAstage0 + kS32 * kAcolsStage <= kTmemCols, "tensor memory budget");
 static_assert(kStageBytesP % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(2 * (kSmemP + 1024) > 228 * 1024, "the ring must keep the kernel at one CTA per SM");
 static_assert(kSmemP <= 227 * 1024, "shared memory per CTA");
 
 struct PipeBars {
-  u64 full[kS32], empty[kS32], afull[kSA], aempty[kSA], accf;
+  u64 full[kS32], afull[kS32], aempty[kS32], accf[2], accfree[2], drain;
 };
 
 __device__ __forceinline__ void mbar_arrive(uint32_t addr) {
@@ -475,12 +484,14 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // MODE 0: P = R (W V), A rows = rows of R, K = columns (tile box 32 x 128,
 //         128-byte swizzle: 16-byte group g of tile row r sits at g ^ (r % 8)).
 // MODE 1: Q^T = R^T U, A rows = columns of R, K = rows (box 128 x 32, no swizzle).
-// Bop: ternary B chunks of the K range, 4 KB per 32 K entries (umma_layout.cuh).
+// T tiles of 128 output rows, C chunks of 32 along K, U = T C units over
+// gridDim.x CTAs; S = slots per tile of Xp (umma_layout.cuh).
+// Bop: ternary B chunks of the K range, 4 KB per 32 K entries.
 // wpad: for MODE 0 the weights, zero padded to a multiple of 32 (or null).
 template <int MODE>
 __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
     const __grid_constant__ CUtensorMap tmap, int m, int n, const unsigned char* __restrict__ Bop,
-    const float* __restrict__ wpad, int bb, int klen, float* __restrict__ Xp,
+    const float* __restrict__ wpad, int bb, int C, long long U, int S, float* __restrict__ Xp,
     int* __restrict__ status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -488,10 +499,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int M = MODE == 0 ? m : n, Kdim = MODE == 0 ? n : m;
-  const int i0 = blockIdx.x * kM, split = blockIdx.y;
-  const int k_begin = split * klen, k_end = min(Kdim, k_begin + klen);
-  const int nchunks = k_end > k_begin ? (k_end - k_begin + kKc - 1) / kKc : 0;
+  const int G = gridDim.x, b = blockIdx.x;
+  const int M = MODE == 0 ? m : n;
+  const long long u0 = sk_u0(b, U, G), u1 = sk_u0(b + 1, U, G);
+  const int nunits = (int)(u1 - u0);
   const bool weighted = MODE == 0 && wpad != nullptr;
   volatile int* ab = &abort_flag;
 
@@ -502,13 +513,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
   if (tid == 32) {
     for (int s = 0; s < kS32; ++s) {
       mbar_init(smem_u32(&bars.full[s]), 1);
-      mbar_init(smem_u32(&bars.empty[s]), 8);
-    }
-    for (int s = 0; s < kSA; ++s) {
       mbar_init(smem_u32(&bars.afull[s]), 8);
       mbar_init(smem_u32(&bars.aempty[s]), 1);
     }
-    mbar_init(smem_u32(&bars.accf), 1);
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(smem_u32(&bars.accf[q]), 1);
+      mbar_init(smem_u32(&bars.accfree[q]), kEpiWarps);
+    }
+    mbar_init(smem_u32(&bars.drain), 1);
     fence_mbar_init();
     abort_flag = 0;
   }
@@ -521,56 +533,120 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
     if (lane == 0) {  // ---- producer ----
       const uint32_t tx = kTileBytes32 + kBBytes + (weighted ? kKc * 4 : 0);
       int issued = 0;
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % kS32;
-        if (c >= kS32 && !mbar_wait_ab(smem_u32(&bars.empty[s]), ((c / kS32) + 1) & 1, ab))
+      // (tile, chunk) of the current unit, advanced incrementally: a 64-bit
+      // division per chunk would cost more than the chunk's MMAs
+      int t = (int)(u0 / C), c = (int)(u0 - (long long)t * C);
+      for (int i = 0; i < nunits; ++i, c = (c + 1 == C) ? 0 : c + 1, t += (c == 0) ? 1 : 0) {
+        const int s = i % kS32;
+        // stage s (fp32 tile, B, A in tensor memory) is free once the MMAs
+        // of chunk i - kS32 have completed
+        if (i >= kS32 && !mbar_wait_ab(smem_u32(&bars.aempty[s]), ((i / kS32) + 1) & 1, ab))
           break;
+        const int kk = c * kKc;
         const uint32_t fb = smem_u32(&bars.full[s]);
         const uint32_t dst = smem_u32(ring + s * kStageBytesP);
-        const int kk = k_begin + c * kKc;
         mbar_expect_tx(fb, tx);
         if (MODE == 0)
-          tma_load_2d(dst, &tmap, kk, i0, fb);
+          tma_load_2d(dst, &tmap, kk, t * kM, fb);
         else
-          tma_load_2d(dst, &tmap, i0, kk, fb);
+          tma_load_2d(dst, &tmap, t * kM, kk, fb);
         bulk_load(dst + kBOff, Bop + (size_t)(kk / kKc) * kBBytes, kBBytes, fb);
         if (weighted) bulk_load(dst + kWOff, wpad + kk, kKc * 4, fb);
         ++issued;
       }
       // every issued copy must have landed before the CTA may exit
-      for (int c = issued > kS32 ? issued - kS32 : 0; c < issued; ++c)
-        mbar_wait(smem_u32(&bars.full[c % kS32]), (uint32_t)((c / kS32) & 1));
+      for (int i = issued > kS32 ? issued - kS32 : 0; i < issued; ++i)
+        mbar_wait(smem_u32(&bars.full[i % kS32]), (uint32_t)((i / kS32) & 1));
     }
   } else if (wid == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
       const uint32_t idesc = make_idesc(0);
-      for (int c = 0; c < nchunks; ++c) {
-        const int s = c % kSA;
-        if (!mbar_wait_ab(smem_u32(&bars.afull[s]), (c / kSA) & 1, ab)) break;
+      int seg = 0;
+      bool ok = true;
+      int c = (int)(u0 % C);  // chunk of the current unit within its tile
+      for (int i = 0; i < nunits && ok; ++i, c = (c + 1 == C) ? 0 : c + 1) {
+        const bool first = i == 0 || c == 0;
+        const bool last = i == nunits - 1 || c == C - 1;
+        const int q = seg & 1;
+        // the accumulator of segment seg - 2 must have been read out
+        if (first && seg >= 2 &&
+            !mbar_wait_ab(smem_u32(&bars.accfree[q]), ((seg >> 1) - 1) & 1, ab)) {
+          ok = false;
+          break;
+        }
+        const int s = i % kS32;
+        if (!mbar_wait_ab(smem_u32(&bars.afull[s]), (i / kS32) & 1, ab)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t acol = tmem + kN + s * kAcolsStage;
-        const uint32_t bbase = smem_u32(ring + kBRingOff + s * kBBytes);
+        const uint32_t acc = tmem + kAcc0 + q * kN;
+        const uint32_t acol = tmem + kAstage0 + s * kAcolsStage;
+        const uint32_t bbase = smem_u32(ring + s * kStageBytesP + kBOff);
 #pragma unroll
         for (int p = 0; p < 3; ++p)
 #pragma unroll
           for (int ks = 0; ks < kKc / 16; ++ks)
-            umma_ts_bf16(tmem, acol + p * (kKc / 2) + ks * 8,
-                         make_desc(bbase + ks * 256, 128, kSboK), idesc,
-                         (c > 0 || p > 0 || ks > 0) ? 1u : 0u);
+            umma_ts_bf16(acc, acol + p * (kKc / 2) + ks * 8, make_desc(bbase + ks * 256, 128, kSboK),
+                         idesc, (!first || p > 0 || ks > 0) ? 1u : 0u);
         umma_commit(smem_u32(&bars.aempty[s]));
+        if (last) {
+          umma_commit(smem_u32(&bars.accf[q]));
+          ++seg;
+        }
       }
       // completes once every MMA issued above has finished (also after an abort)
-      umma_commit(smem_u32(&bars.accf));
+      umma_commit(smem_u32(&bars.drain));
+      mbar_wait(smem_u32(&bars.drain), 0u);
+    }
+  } else if (wid < kConvWarp0) {
+    // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31, all 64 columns ----
+    const int quad = wid & 3;
+    const int t_first = nunits > 0 ? (int)(u0 / C) : 0;
+    const int nsegs = nunits > 0 ? (int)((u1 - 1) / C) - t_first + 1 : 0;
+    for (int sg = 0; sg < nsegs; ++sg) {
+      const int q = sg & 1;
+      const bool ok = mbar_wait_ab(smem_u32(&bars.accf[q]), (sg >> 1) & 1, ab);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int t = t_first + sg;
+      const int slot = b - sk_first(t, C, U, G);
+      const int row = quad * 32 + lane, gi = t * kM + row;
+      float* out = Xp + ((size_t)((size_t)t * S + slot) * kM + row) * bb;
+#pragma unroll
+      for (int h = 0; h < kN / 16; ++h) {
+        uint32_t v[16];
+        tmem_ld16(tmem + kAcc0 + q * kN + ((uint32_t)(quad * 32) << 16) + (uint32_t)(h * 16), v);
+        if (gi < M) {
+          if (bb == kN) {
+#pragma unroll
+            for (int t4 = 0; t4 < 4; ++t4)
+              *(float4*)(out + h * 16 + 4 * t4) =
+                  make_float4(__uint_as_float(v[4 * t4]), __uint_as_float(v[4 * t4 + 1]),
+                              __uint_as_float(v[4 * t4 + 2]), __uint_as_float(v[4 * t4 + 3]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              if (h * 16 + e < bb) out[h * 16 + e] = __uint_as_float(v[e]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars.accfree[q]));
     }
   } else {
-    // ---- converters (warps 2..9) ----
-    const int quad = wid & 3;          // TMEM lanes this warp may access
-    const int kh = (wid - 2) >> 2;     // K half of each chunk
-    const int row = quad * 32 + lane;  // tile row = TMEM lane
-    const int ctid = tid - 64;         // 0..255: one 16-byte piece of B
-    for (int c = 0; c < nchunks; ++c) {
-      const int s = c % kS32, sa = c % kSA;
-      bool ok = mbar_wait_ab(smem_u32(&bars.full[s]), (c / kS32) & 1, ab);
+    // ---- converters (two groups of eight warps, alternate chunks) ----
+    const int cw = wid - kConvWarp0;
+    const int grp = cw >> 3;
+    const int quad = wid & 3;               // TMEM lanes this warp may access
+    const int kh = (cw >> 2) & 1;           // K half of each chunk
+    const int row = quad * 32 + lane;       // tile row = TMEM lane
+    for (int i = grp; i < nunits; i += kConvGroups) {
+      const int s = i % kS32;
+      // the copies of chunk i have landed; the producer waited for the MMAs of
+      // chunk i - kS32 before issuing them, so A stage s is free as well
+      const bool ok = mbar_wait_ab(smem_u32(&bars.full[s]), (i / kS32) & 1, ab);
       if (!__all_sync(0xffffffffu, ok)) break;
       const unsigned char* st = ring + s * kStageBytesP;
       float x[16];
@@ -593,9 +669,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
 #pragma unroll
         for (int e = 0; e < 16; ++e) x[e] = *(const float*)(st + (kh * 16 + e) * 512 + row * 4);
       }
-      const uint4 bpiece = *(const uint4*)(st + kBOff + ctid * 16);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.empty[s]));  // the fp32 stage is free again
       uint32_t ph[8], pm[8], pl[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -606,41 +679,16 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
         pm[e] = pack2(m0, m1);
         pl[e] = pack2(l0, l1);
       }
-      // A / B stage sa: the MMAs of chunk c - kSA must be done with it
-      ok = c < kSA || mbar_wait_ab(smem_u32(&bars.aempty[sa]), ((c / kSA) + 1) & 1, ab);
-      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + kN + sa * kAcolsStage + kh * 8;
+      const uint32_t ta =
+          tmem + ((uint32_t)(quad * 32) << 16) + kAstage0 + s * kAcolsStage + kh * 8;
       tmem_st8(ta, ph);
       tmem_st8(ta + kKc / 2, pm);
       tmem_st8(ta + kKc, pl);
-      *(uint4*)(ring + kBRingOff + sa * kBBytes + ctid * 16) = bpiece;
       tmem_st_wait();
-      fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars.afull[sa]));
-    }
-    // ---- epilogue: accumulator columns 32 kh .. 32 kh + 31 of lane `row` ----
-    mbar_wait(smem_u32(&bars.accf), 0u);
-    tc_fence_after();
-    const int gi = i0 + row;
-    float* out = Xp + ((size_t)split * M + gi) * bb;
-    if (nchunks == 0) {
-      if (gi < M)
-        for (int t = 0; t < 32; ++t)
-          if (kh * 32 + t < bb) out[kh * 32 + t] = 0.f;
-    } else if (!*ab) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t v[16];
-        const int col = kh * 32 + h * 16;
-        tmem_ld16(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)col, v);
-        if (gi < M)
-#pragma unroll
-          for (int t = 0; t < 16; ++t)
-            if (col + t < bb) out[col + t] = __uint_as_float(v[t]);
-      }
+      if (lane == 0) mbar_arrive(smem_u32(&bars.afull[s]));
     }
   }
   tc_fence_before();
@@ -710,39 +758,62 @@ void set_attrs() {
 
 }  // namespace
 
-// Host launchers; klen must be a multiple of kKc (32).  Rows of R that start
-// 16-byte aligned take the TMA-pipelined kernel, others the direct-load one.
+// Stream-K plan of a contraction with M output rows and K-dimension Kdim:
+// G CTAs (at most one per SM, and few enough that no tile is split into more
+// than kMaxSegs segments), S = most segments of any tile.
+void tc_contract_plan(int M, int Kdim, int nsm, TcPlan* p) {
+  using namespace umma;
+  p->T = (M + kM - 1) / kM;
+  p->C = (Kdim + kKc - 1) / kKc;
+  p->U = (long long)p->T * p->C;
+  long long g = std::min<long long>(nsm, p->U);
+  g = std::min<long long>(g, (long long)(kMaxSegs - 1) * p->T);
+  p->G = (int)std::max<long long>(1, g);
+  p->S = 1;
+  for (int t = 0; t < p->T; ++t) p->S = std::max(p->S, sk_nseg(t, p->C, p->U, p->G));
+}
+
+// rows of an n-column fp32 matrix at a 16-byte aligned base are TMA-addressable
+bool tc_contract_tma_ok(int n) { return tma_ok(nullptr, n) && encode_fn() != nullptr; }
+
+// Host launchers.  With a plan the TMA kernel runs and writes stream-K tile
+// partials (callers check tc_contract_tma_ok first); without one the direct
+// kernel writes `splits` split-K partials over K ranges of klen (a multiple
+// of 32).
 int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
                    const unsigned long long* Vs, const unsigned char* Bop, const float* w,
-                   const float* wpad, int bb, int klen, int splits, float* Pp, cudaStream_t st) {
+                   const float* wpad, int bb, const TcPlan* p, int klen, int splits, float* Pp,
+                   cudaStream_t st) {
   using namespace umma;
   set_attrs();
   int* status = status_word_ptr();
-  dim3 grid((unsigned)((m + kM - 1) / kM), (unsigned)splits);
   CUtensorMap tm;
-  if (tma_ok(R, n) && make_tmap(&tm, R, m, n, 0))
-    contract_tma_kernel<0><<<grid, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, w ? wpad : nullptr,
-                                                            bb, klen, Pp, status);
-  else
-    contract_kernel<0><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Vm, Vs, w, bb, klen, Pp,
-                                                                 status);
+  if (p) {
+    if (!make_tmap(&tm, R, m, n, 0)) return EXTERND_ERR_CUDA;
+    contract_tma_kernel<0><<<p->G, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, w ? wpad : nullptr, bb,
+                                                            p->C, p->U, p->S, Pp, status);
+  } else {
+    contract_kernel<0><<<dim3((unsigned)((m + kM - 1) / kM), (unsigned)splits), umma::kThreads,
+                         kSmemBytes, st>>>(R, m, n, Vm, Vs, w, bb, klen, Pp, status);
+  }
   return cudaGetLastError() == cudaSuccess ? EXTERND_OK : EXTERND_ERR_CUDA;
 }
 
 int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
-                    const unsigned long long* Us, const unsigned char* Bop, int bb, int klen,
-                    int splits, float* Qp, cudaStream_t st) {
+                    const unsigned long long* Us, const unsigned char* Bop, int bb, const TcPlan* p,
+                    int klen, int splits, float* Qp, cudaStream_t st) {
   using namespace umma;
   set_attrs();
   int* status = status_word_ptr();
-  dim3 grid((unsigned)((n + kM - 1) / kM), (unsigned)splits);
   CUtensorMap tm;
-  if (tma_ok(R, n) && make_tmap(&tm, R, m, n, 1))
-    contract_tma_kernel<1><<<grid, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, nullptr, bb, klen, Qp,
-                                                            status);
-  else
-    contract_kernel<1><<<grid, umma::kThreads, kSmemBytes, st>>>(R, m, n, Um, Us, nullptr, bb,
-                                                                 klen, Qp, status);
+  if (p) {
+    if (!make_tmap(&tm, R, m, n, 1)) return EXTERND_ERR_CUDA;
+    contract_tma_kernel<1><<<p->G, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, nullptr, bb, p->C, p->U,
+                                                            p->S, Qp, status);
+  } else {
+    contract_kernel<1><<<dim3((unsigned)((n + kM - 1) / kM), (unsigned)splits), umma::kThreads,
+                         kSmemBytes, st>>>(R, m, n, Um, Us, nullptr, bb, klen, Qp, status);
+  }
   return cudaGetLastError() == cudaSuccess ? EXTERND_OK : EXTERND_ERR_CUDA;
 }
 

@@ -44,3 +44,33 @@ __device__ __forceinline__ uint4 bf16_codes8(uint32_t m8, uint32_t s8) {
 
 }  // namespace umma
 }  // namespace externd
+
+namespace externd {
+namespace umma {
+
+// Stream-K partition of a contraction: the (tile, K-chunk) units u = t C + c
+// (T tiles of 128 output rows, C chunks of 32 along K) are split into G
+// contiguous ranges [u0(b), u0(b+1)), one per CTA.  A CTA's range covers a
+// run of tiles; its part of tile t is one "segment" with its own partial
+// result.  The segments of a tile belong to consecutive CTAs
+// first(t) .. last(t), and CTA b's partial of tile t goes to slot
+// b - first(t) of that tile: Xp[(t * S + slot) * 128 + row][64] (S = most
+// segments of any tile).  A tile's partials are summed in slot order.
+__host__ __device__ __forceinline__ long long sk_u0(int b, long long U, int G) {
+  return (long long)b * U / G;
+}
+__host__ __device__ __forceinline__ int sk_owner(long long u, long long U, int G) {
+  int b = (int)((u * G) / U);
+  while (b + 1 < G && sk_u0(b + 1, U, G) <= u) ++b;
+  while (b > 0 && sk_u0(b, U, G) > u) --b;
+  return b;
+}
+__host__ __device__ __forceinline__ int sk_first(int t, int C, long long U, int G) {
+  return sk_owner((long long)t * C, U, G);
+}
+__host__ __device__ __forceinline__ int sk_nseg(int t, int C, long long U, int G) {
+  return sk_owner((long long)(t + 1) * C - 1, U, G) - sk_first(t, C, U, G) + 1;
+}
+
+}  // namespace umma
+}  // namespace externd
