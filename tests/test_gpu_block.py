@@ -115,3 +115,24 @@ def test_block_deterministic():
     for a, b in ((f1.packed_B, f2.packed_B), (f1.packed_C, f2.packed_C), (f1.D, f2.D),
                  (f1.energy, f2.energy)):
         assert torch.equal(a, b)
+
+
+def test_transformer_block_weighted(oracle):
+    """The seven importance-weighted matrices of one transformer block (mu = 3,
+    b = 64): the first block of q teacher-forced, every matrix free-running
+    against the oracle's stored final energy."""
+    wls = W.config_block_matrices(64)
+    q = wls[0]
+    rep, f = block_teacher_forced(oracle, q.a, q.mu, q.tau, q.iters, 64, blocks=[0], w=q.w)
+    print(f"block_q b=64 weighted: band {rep.band_total} mismatch {rep.band_mismatch} "
+          f"max D rel {rep.d_rel_max:.2e}")
+    assert rep.ok, rep.bad
+    p = os.path.join(os.path.dirname(__file__), "golden", "oracle_energy.json")
+    g = json.load(open(p))
+    for wl in wls:
+        ref = g[wl.name]
+        assert ref["k"] == wl.k and ref["block"] == 64
+        fw = X.decompose(_dev(wl.a), wl.mu, wl.tau, wl.iters, block=64, w=_dev(wl.w))
+        e = float(fw.energy[-1])
+        print(f"  {wl.name} {wl.m}x{wl.n}: device {e:.8f} oracle {ref['final_energy']:.8f}")
+        assert abs(e - ref["final_energy"]) <= FREE_ENERGY_ATOL
