@@ -33,6 +33,10 @@ MUTATIONS = [
      "return tr > 0.0 ? 1e-1 * tr / (double)b : 1.0;"),
     ("block_closed_form_sign", "e -= 2.0 * (double)dl[a] * r[a];", "e += 2.0 * (double)dl[a] * r[a];"),
     ("safeguard_keeps_u", "std::fill(u.begin(), u.end(), 0);", ";"),
+    ("block_gram_unweighted", "s += wt(w, j) * V[l * n + j] * V[l2 * n + j];",
+     "s += V[l * n + j] * V[l2 * n + j];"),
+    ("block_u_target_unweighted", "s += (double)R[i * n + j] * wt(w, j) * V[l * n + j];",
+     "s += (double)R[i * n + j] * V[l * n + j];"),
 ]
 
 PIN_TESTS = [
@@ -49,6 +53,8 @@ PIN_TESTS = [
     pins.test_reconstruct_matches_matmul_and_energy,
     pins.test_weighted_energy_is_weighted_norm,
     pins.test_block_scales_solve_normal_equations,
+    lambda o: pins.test_block_targets_solve_their_normal_equations(o, False),
+    lambda o: pins.test_block_targets_solve_their_normal_equations(o, True),
     pins.test_block_energy_matches_replay,
     pins.test_exact_recovery_of_ternary_rank1,
     pins.test_exact_recovery_of_two_disjoint_components,

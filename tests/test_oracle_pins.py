@@ -334,3 +334,39 @@ def test_exact_recovery_of_two_disjoint_components(oracle):
     assert dec.energy[0] == pytest.approx(e1 / (e1 + e2), rel=1e-15)
     assert dec.energy[1] == 1.0
     assert abs(dec.D[0]) == 2.0 and abs(dec.D[1]) == 0.5
+
+
+@pytest.mark.parametrize("weighted", [False, True])
+def test_block_targets_solve_their_normal_equations(oracle, weighted):
+    """Block-ALS half-steps (b > 1): the U target T solves T (V^T W V + eps I) = R W V
+    and the V target solves (U^T U + eps I) T^T = U^T R (Eq. (3), eps = 1e-6 tr(G)/b);
+    every code is the sign of its target entry where |T| exceeds its column's
+    tau * rms threshold, else 0."""
+    rng = np.random.default_rng(17)
+    m, n, b, tau = 37, 29, 5, 0.5
+    R = (rng.standard_normal((m, n)) * 0.1).astype(np.float32)
+    w = rng.lognormal(0.0, 1.0, n).astype(np.float32) if weighted else None
+    V = rng.integers(-1, 2, size=(b, n)).astype(np.int8)
+    V[:, 0] = 1  # no empty component
+    U, T, thr = oracle.block_u_step(R, V, tau, w)
+    Wd = np.diag(w.astype(np.float64)) if weighted else np.eye(n)
+    Vt = V.T.astype(np.float64)
+    G = Vt.T @ Wd @ Vt
+    eps = 1e-6 * np.trace(G) / b
+    lhs = T @ (G + eps * np.eye(b))
+    rhs = R.astype(np.float64) @ Wd @ Vt
+    assert np.abs(lhs - rhs).max() <= 1e-10 * np.abs(rhs).max()
+    rms = np.sqrt((T * T).mean(axis=0))
+    np.testing.assert_allclose(thr, tau * rms, rtol=1e-12)
+    want = np.where(np.abs(T) > thr, np.sign(T), 0).astype(np.int8).T
+    assert np.array_equal(U, want)
+
+    V2, T2, thr2 = oracle.block_v_step(R, U, tau)
+    Ut = U.T.astype(np.float64)
+    GU = Ut.T @ Ut
+    epsU = 1e-6 * np.trace(GU) / b if np.trace(GU) > 0 else 1.0
+    lhs2 = (GU + epsU * np.eye(b)) @ T2.T
+    rhs2 = Ut.T @ R.astype(np.float64)
+    assert np.abs(lhs2 - rhs2).max() <= 1e-10 * max(np.abs(rhs2).max(), 1e-300)
+    want2 = np.where(np.abs(T2) > thr2, np.sign(T2), 0).astype(np.int8).T
+    assert np.array_equal(V2, want2)
