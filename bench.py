@@ -274,6 +274,10 @@ def run_ours(args, rank, world, local_rank):
              torch.empty(o.D.shape, dtype=torch.float32).pin_memory(),
              torch.empty(o.energy.shape, dtype=torch.float64).pin_memory()) for o in outs]
     A2s = [torch.empty_like(A) for A in As]
+    for A2, hA in zip(A2s, hAs):
+        A2.copy_(hA, non_blocking=True)
+    for _ in range(max(args.warmup, 0)):  # untimed: the same calls as the timed ones
+        step(A2s)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     if world > 1:

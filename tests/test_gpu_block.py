@@ -136,3 +136,33 @@ def test_transformer_block_weighted(oracle):
         e = float(fw.energy[-1])
         print(f"  {wl.name} {wl.m}x{wl.n}: device {e:.8f} oracle {ref['final_energy']:.8f}")
         assert abs(e - ref["final_energy"]) <= FREE_ENERGY_ATOL
+
+
+def test_graph_replay_matches_direct(monkeypatch):
+    """Repeated identical calls are replayed from a captured CUDA graph (the
+    first runs directly, the second captures); the replayed results equal a
+    direct run bit for bit, also when A's contents change between calls."""
+    A = _dev(W.llm_like(640, 512, 21, n_outliers=2))
+    A0 = A.clone()
+    k = X.rank(640, 512, 0.5)
+    f = X.alloc_factors(640, 512, k, A.device)
+    outs = []
+    for _ in range(3):  # direct, capture + replay, replay
+        X.decompose_into(f, A, 0.5, 0.5, 3, block=32)
+        outs.append([t.clone() for t in (f.packed_B, f.packed_C, f.D, f.energy)])
+    A.mul_(1.5)  # new contents under the same pointer: the replay must see them
+    X.decompose_into(f, A, 0.5, 0.5, 3, block=32)
+    scaled = [t.clone() for t in (f.packed_B, f.packed_C, f.D, f.energy)]
+    assert X.sync_status() == X.OK
+    monkeypatch.setenv("EXTERND_NO_GRAPH", "1")
+    g = X.alloc_factors(640, 512, k, A.device)
+    X.decompose_into(g, A, 0.5, 0.5, 3, block=32)
+    direct_scaled = [t.clone() for t in (g.packed_B, g.packed_C, g.D, g.energy)]
+    A.copy_(A0)
+    X.decompose_into(g, A, 0.5, 0.5, 3, block=32)
+    direct = [g.packed_B, g.packed_C, g.D, g.energy]
+    for run in outs:
+        for a, b in zip(run, direct):
+            assert torch.equal(a, b)
+    for a, b in zip(scaled, direct_scaled):
+        assert torch.equal(a, b)
