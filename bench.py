@@ -173,7 +173,7 @@ def _profiled_traffic(kernel: str, workload: str):
         if ent.get("workload") != workload:
             return None
         from expanded_rank_matrix_b200 import build as B
-        if ent.get("source_hash") != B.source_hash():
+        if ent.get("kernel_source_hash") != B.kernel_source_hash(kernel):
             return None
         return ent.get("dram_bytes_per_launch")
     except Exception:  # noqa: BLE001

@@ -51,6 +51,24 @@ if __name__ == "__main__":
     print(build(force=True, verbose="-v" in sys.argv))
 
 
+# the source files each profiled kernel is built from
+KERNEL_SOURCES = {
+    "seq_als_kernel": ("seq_als.cu", "common.cuh"),
+    "contract_tma_kernel": ("umma_contract.cu", "umma_layout.cuh", "common.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the files one kernel is compiled from (identifies that kernel's
+    code across unrelated changes elsewhere in the library)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(name.encode())
+        h.update(open(os.path.join(CSRC, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def source_hash() -> str:
     """Hash of the CUDA sources and the public header (identifies a kernel build)."""
     import hashlib
