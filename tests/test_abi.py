@@ -74,6 +74,26 @@ def test_host_argument_checks(lib):
                                       nul, nul, nul, nul, nul, -1, nul) == X.ERR_INVALID_ARG
 
 
+def test_block_argument_checks(lib):
+    L = lib
+    nul = None
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected before any CUDA call
+    # block-ALS: at most 64 components per block, and no more than k or min(m, n)
+    assert L.externd_decompose(fake, 4096, 4096, 1.0, 0.5, 2, nul, 65, fake, fake, fake, fake,
+                               nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose(fake, 40, 30, 1.0, 0.5, 2, nul, 31, fake, fake, fake, fake,
+                               nul) == X.ERR_INVALID_ARG
+    # the block-traced entry is block-mode only and needs its trace buffers
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 1, fake, fake, fake,
+                                            fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, fake, fake, fake,
+                                            fake, 2, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, fake, fake, fake,
+                                            fake, -1, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 65, fake, fake, fake,
+                                            fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+
+
 def test_unpack_planes_layout():
     import numpy as np
     # entries: +1 at 0, -1 at 1, 0 at 2, +1 at 33 (second word)
