@@ -759,14 +759,18 @@ void set_attrs() {
 }  // namespace
 
 // Stream-K plan of a contraction with M output rows and K-dimension Kdim:
-// G CTAs (at most one per SM, and few enough that no tile is split into more
+// G CTAs (one per SM but one, and few enough that no tile is split into more
 // than kMaxSegs segments), S = most segments of any tile.
 void tc_contract_plan(int M, int Kdim, int nsm, TcPlan* p) {
   using namespace umma;
   p->T = (M + kM - 1) / kM;
   p->C = (Kdim + kKc - 1) / kKc;
   p->U = (long long)p->T * p->C;
-  long long g = std::min<long long>(nsm, p->U);
+  // one SM is left to the Gram / inverse kernels that run beside the
+  // contraction on a side stream: they cannot share an SM with a contraction
+  // CTA (registers), so on a full grid one CTA, and with it the launch, would
+  // wait for them (17 % of a 9728 x 2560 block-ALS decomposition)
+  long long g = std::min<long long>(nsm > 1 ? nsm - 1 : 1, p->U);
   g = std::min<long long>(g, (long long)(kMaxSegs - 1) * p->T);
   p->G = (int)std::max<long long>(1, g);
   p->S = 1;
