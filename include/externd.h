@@ -88,6 +88,18 @@ int64_t externd_rank(int64_t m, int64_t n, float mu);
  *   stream       CUDA stream (NULL = legacy default stream).
  * Returns EXTERND_OK or a negative status.  On a device-detected error the
  * outputs are undefined and externd_sync_status() returns the error.
+ *
+ * Scratch: the call allocates its workspace stream-ordered on `stream`
+ * (cudaMallocAsync) and frees it before the work it queued completes.
+ * Block mode replays repeated calls: a call whose pointers, sizes and knobs
+ * equal an earlier call's on the same device (the second such call) is
+ * captured once into a CUDA graph on a library-owned stream and replayed
+ * from then on, joined to `stream` by events; the library keeps up to 8
+ * such graphs (least recently used first out), whose workspace lives in the
+ * device's graph memory pool.  The replay reads A and w at launch time, so
+ * new contents under the same pointers are honoured.  Calls on a stream that
+ * is being captured run directly (they become part of the caller's graph);
+ * setting the environment variable EXTERND_NO_GRAPH=1 disables replay.
  */
 int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
                       const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
