@@ -770,9 +770,7 @@ void tc_contract_plan(int M, int Kdim, int nsm, TcPlan* p) {
   // contraction on a side stream: they cannot share an SM with a contraction
   // CTA (registers), so on a full grid one CTA, and with it the launch, would
   // wait for them (17 % of a 9728 x 2560 block-ALS decomposition)
-  long long g = std::min<long long>(nsm > 1 ? nsm - 1 : 1, p->U);
-  g = std::min<long long>(g, (long long)(kMaxSegs - 1) * p->T);
-  p->G = (int)std::max<long long>(1, g);
+  p->G = sk_ctas(p->T, p->C, nsm, kMaxSegs);
   p->S = 1;
   for (int t = 0; t < p->T; ++t) p->S = std::max(p->S, sk_nseg(t, p->C, p->U, p->G));
 }

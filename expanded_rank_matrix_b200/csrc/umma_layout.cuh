@@ -72,5 +72,17 @@ __host__ __device__ __forceinline__ int sk_nseg(int t, int C, long long U, int G
   return sk_owner((long long)(t + 1) * C - 1, U, G) - sk_first(t, C, U, G) + 1;
 }
 
+// CTA count of a contraction with T tiles and C chunks on nsm SMs: one CTA
+// per SM but one (that SM runs the kernels beside the contraction), at most
+// one per unit, and few enough that no tile has more than max_segs segments
+// (G <= (max_segs - 1) T gives at least C / (max_segs - 1) units per CTA).
+inline int sk_ctas(int T, int C, int nsm, int max_segs) {
+  long long g = (long long)T * C;
+  const long long cap = nsm > 1 ? nsm - 1 : 1;
+  if (cap < g) g = cap;
+  if ((long long)(max_segs - 1) * T < g) g = (long long)(max_segs - 1) * T;
+  return g < 1 ? 1 : (int)g;
+}
+
 }  // namespace umma
 }  // namespace externd
