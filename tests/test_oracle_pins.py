@@ -176,6 +176,43 @@ def test_safeguard_zeroes_best_entry(oracle):
     assert dec.energy[-1] == 1.0 - oracle.sumsq(R) / oracle.sumsq(A)
 
 
+def test_weighted_safeguard_takes_largest_weighted_square(oracle):
+    """Weighted single-entry step ([PITH] Appendix A, Prop. 2 under the weighted
+    norm of Sec. 2.5): with tau so large that every ALS pair is empty, each
+    component is the entry of largest w_j R_ij^2 -- scored in fp32 as
+    (R_ij * R_ij) * w_j, ties to the lowest row-major index -- and that entry
+    is zeroed exactly.  The weights are spread so that the weighted and the
+    unweighted argmax differ, and a planted tie checks the index rule."""
+    rng = _rng(19)
+    m, n = 11, 9
+    A = rng.standard_normal((m, n)).astype(np.float32)
+    w = np.exp(2.0 * rng.standard_normal(n)).astype(np.float32)
+    # a tie in the weighted score: same |value| in the same column, two rows
+    A[7, 4] = np.float32(9.0)
+    A[2, 4] = np.float32(-9.0)
+    w[4] = np.float32(50.0)
+    k = 6
+    dec = oracle.decompose(A, k, 100.0, 2, w=w)
+    assert dec.n_fallback == k and dec.fallback.all()
+    R = A.copy()
+    differs = 0
+    for c in range(k):
+        score = (R * R).astype(np.float32) * w[None, :]   # fp32 products, as the reading fixes
+        flat = int(np.argmax(score))                       # first maximum = lowest row-major index
+        i, j = divmod(flat, n)
+        differs += int(flat != int(np.argmax(np.abs(R))))
+        assert dec.U[c].tolist() == [1 if t == i else 0 for t in range(m)], c
+        assert dec.V[c].tolist() == [1 if t == j else 0 for t in range(n)], c
+        assert dec.D[c] == R[i, j]
+        if c == 0:
+            assert (i, j) == (2, 4)  # the tie goes to the lower row
+        f2, M = oracle.entry_max(R, w)
+        assert f2 == flat and M == float(score.reshape(-1)[flat])
+        R = oracle.replay(A, dec.U, dec.V, dec.D, c + 1)
+        assert R[i, j] == 0.0
+    assert differs >= 1  # the weights changed at least one choice
+
+
 @pytest.mark.parametrize("tau", [0.5, 100.0])
 def test_prop2_geometric_bound(oracle, tau):
     rng = _rng(31)
