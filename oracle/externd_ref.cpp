@@ -19,8 +19,18 @@
 //
 // Readings taken where the pages leave a step open (each is listed in the
 // design notes with its reason):
-//   * T_tau(x)_j = sign(x_j) if |x_j| > tau * rms(x) else 0; rms over the
-//     whole vector, computed in fp64; strict comparison.
+//   * T_tau(x)_j = sign(x_j) if |x_j| > tau * s(x) else 0, strict, with the
+//     statistic s computed in fp64 over the whole vector: s = rms(x) by
+//     default; s = mean |x| in the threshold variant ([REV] "Method" quotes
+//     zero shares, tau = 0.7 -> ~41% and tau = 2.0 -> ~87%, that a mean-|x|
+//     statistic reproduces on Gaussian data and rms does not).
+//   * Naive weighted V-step (the ablation [REV] "Validation" names):
+//     v = T_tau(W R^T u); the default (corrected) V-step thresholds R^T u.
+//   * Refinement sweeps (backfitting, [REV] "Results"): component l is added
+//     back onto the residual and refit by ALS from its own v; the refit
+//     replaces it only if it removes more than the old pattern with its
+//     scale re-solved on that residual, so no sweep step raises the residual;
+//     the single-entry step applies as in the greedy pass.
 //   * The residual R is kept in the input's precision (fp32).  A deflation
 //     R_ij <- R_ij - u_i v_j d is one IEEE fp32 add or subtract of the fp32
 //     scale d (u_i v_j is +-1 or 0), never fused with anything else.
@@ -93,11 +103,13 @@ extern "C" {
 
 // T_tau, the adaptive ternarisation operator ([PITH] Eq. 2 via "Assumptions &
 // free parameters"; [REV] "Method": tau sets the share of zeros).  Writes the
-// ternary codes and returns the threshold tau * rms(x).
-double orc_ternarize(const double* x, int64_t len, double tau, int8_t* out) {
+// ternary codes and returns the threshold tau * s(x), s = rms (stat 0) or
+// mean |x| (stat 1).
+double orc_ternarize2(const double* x, int64_t len, double tau, int stat, int8_t* out) {
   double s = 0.0;
-  for (int64_t j = 0; j < len; ++j) s += x[j] * x[j];
-  double thr = len > 0 ? tau * std::sqrt(s / (double)len) : 0.0;
+  for (int64_t j = 0; j < len; ++j) s += stat == 1 ? std::fabs(x[j]) : x[j] * x[j];
+  double thr = 0.0;
+  if (len > 0) thr = stat == 1 ? tau * (s / (double)len) : tau * std::sqrt(s / (double)len);
   for (int64_t j = 0; j < len; ++j) {
     double a = std::fabs(x[j]);
     out[j] = (a > thr) ? (x[j] > 0.0 ? 1 : -1) : 0;
@@ -105,10 +117,14 @@ double orc_ternarize(const double* x, int64_t len, double tau, int8_t* out) {
   return thr;
 }
 
+double orc_ternarize(const double* x, int64_t len, double tau, int8_t* out) {
+  return orc_ternarize2(x, len, tau, 0, out);
+}
+
 // ALS u half-step ([PITH] referee summary, Sec. 2.3: ternarise against the
 // current residual): y = R (w o v), u = T_tau(y).  Returns the threshold.
-double orc_u_step(const float* R, int64_t m, int64_t n, const int8_t* v, const float* w,
-                  double tau, double* y, int8_t* u) {
+double orc_u_step2(const float* R, int64_t m, int64_t n, const int8_t* v, const float* w,
+                   double tau, int stat, double* y, int8_t* u) {
   for (int64_t i = 0; i < m; ++i) {
     double s = 0.0;
     const float* row = R + i * n;
@@ -116,19 +132,34 @@ double orc_u_step(const float* R, int64_t m, int64_t n, const int8_t* v, const f
       if (v[j]) s += (double)row[j] * ((double)v[j] * wt(w, j));
     y[i] = s;
   }
-  return orc_ternarize(y, m, tau, u);
+  return orc_ternarize2(y, m, tau, stat, u);
 }
 
-// ALS v half-step: z = R^T u, v = T_tau(z).  Returns the threshold.
-double orc_v_step(const float* R, int64_t m, int64_t n, const int8_t* u, double tau,
-                  double* z, int8_t* v) {
+double orc_u_step(const float* R, int64_t m, int64_t n, const int8_t* v, const float* w,
+                  double tau, double* y, int8_t* u) {
+  return orc_u_step2(R, m, n, v, w, tau, 0, y, u);
+}
+
+// ALS v half-step: z = R^T u, v = T_tau(z) -- or, for the naive weighted
+// V-step, v = T_tau(w o z).  z is returned unweighted either way.  Returns
+// the threshold.
+double orc_v_step2(const float* R, int64_t m, int64_t n, const int8_t* u, const float* w,
+                   double tau, int stat, int naive, double* z, int8_t* v) {
   for (int64_t j = 0; j < n; ++j) z[j] = 0.0;
   for (int64_t i = 0; i < m; ++i) {
     if (!u[i]) continue;
     const float* row = R + i * n;
     for (int64_t j = 0; j < n; ++j) z[j] += (double)u[i] * (double)row[j];
   }
-  return orc_ternarize(z, n, tau, v);
+  if (!naive || !w) return orc_ternarize2(z, n, tau, stat, v);
+  std::vector<double> wz(n);
+  for (int64_t j = 0; j < n; ++j) wz[j] = (double)w[j] * z[j];
+  return orc_ternarize2(wz.data(), n, tau, stat, v);
+}
+
+double orc_v_step(const float* R, int64_t m, int64_t n, const int8_t* u, double tau,
+                  double* z, int8_t* v) {
+  return orc_v_step2(R, m, n, u, nullptr, tau, 0, 0, z, v);
 }
 
 // Row energies rho_i = sum_j w_j R_ij^2; returns the index of the largest
@@ -222,13 +253,24 @@ void orc_deflate(float* R, int64_t m, int64_t n, const int8_t* u, const int8_t* 
 
 // Greedy sequential-deflation ALS (paper Sec. 2.3 per [PITH]; [REV] "Method"
 // and "Key idea"), with the best-single-entry safeguard of Prop. 2.
+// flags: bit 0 = mean-|x| threshold statistic, bit 1 = naive weighted V-step.
 // Outputs: U k x m and V k x n ternary codes (row c = component c), D[k],
 // energy[k] = 1 - |R_{c+1}|_W^2 / |A|_W^2, init_row[k] (row whose ternarised
 // copy started the component), fallback[k] (1 when the safeguard fired).
-// Returns the number of safeguard activations.
-int64_t orc_decompose_seq(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
-                          const float* w, int8_t* U, int8_t* V, float* D, double* energy,
-                          int64_t* init_row, uint8_t* fallback) {
+// After the greedy pass, `sweeps` refinement sweeps (orc_refine_sweep) run
+// over the k components; sweep_energy[s] (may be NULL when sweeps == 0) is the
+// energy after sweep s and sweep_flags[s*k + l] the step's flags.  energy[]
+// keeps the greedy pass's trace.  Returns the number of safeguard
+// activations of the greedy pass.
+int64_t orc_refine_sweep(float* R, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                         const float* w, int flags, int8_t* U, int8_t* V, float* D,
+                         uint8_t* step_flags);
+
+int64_t orc_decompose_seq2(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                           const float* w, int flags, int sweeps, int8_t* U, int8_t* V, float* D,
+                           double* energy, int64_t* init_row, uint8_t* fallback,
+                           double* sweep_energy, uint8_t* sweep_flags) {
+  const int stat = flags & 1, naive = (flags >> 1) & 1;
   std::vector<float> R(A, A + m * n);
   std::vector<double> rho(m), y(m), z(n), rowd(n);
   std::vector<int8_t> u(m), v(n);
@@ -246,10 +288,10 @@ int64_t orc_decompose_seq(const float* A, int64_t m, int64_t n, int64_t k, doubl
         int64_t istar = orc_row_norms(R.data(), m, n, w, rho.data());
         init_row[c] = istar;
         for (int64_t j = 0; j < n; ++j) rowd[j] = (double)R[istar * n + j];
-        orc_ternarize(rowd.data(), n, tau, v.data());
+        orc_ternarize2(rowd.data(), n, tau, stat, v.data());
         for (int t = 0; t < iters; ++t) {
-          orc_u_step(R.data(), m, n, v.data(), w, tau, y.data(), u.data());
-          orc_v_step(R.data(), m, n, u.data(), tau, z.data(), v.data());
+          orc_u_step2(R.data(), m, n, v.data(), w, tau, stat, y.data(), u.data());
+          orc_v_step2(R.data(), m, n, u.data(), w, tau, stat, naive, z.data(), v.data());
         }
         double sc[6];
         orc_scale(z.data(), u.data(), v.data(), m, n, w, sc);
@@ -283,7 +325,95 @@ int64_t orc_decompose_seq(const float* A, int64_t m, int64_t n, int64_t k, doubl
     init_row[c] = -1;
     fallback[c] = 0;
   }
+  for (int sw = 0; sw < sweeps; ++sw) {
+    orc_refine_sweep(R.data(), m, n, k, tau, iters, w, flags, U, V, D, sweep_flags + sw * k);
+    sweep_energy[sw] = E0 > 0.0 ? 1.0 - orc_sumsq(R.data(), m, n, w) / E0 : 1.0;
+  }
   return nfb;
+}
+
+int64_t orc_decompose_seq(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                          const float* w, int8_t* U, int8_t* V, float* D, double* energy,
+                          int64_t* init_row, uint8_t* fallback) {
+  return orc_decompose_seq2(A, m, n, k, tau, iters, w, 0, 0, U, V, D, energy, init_row, fallback,
+                            nullptr, nullptr);
+}
+
+// One refinement sweep over the k components on the residual R (backfitting;
+// [REV] "Results": sweeps add ~0.4 energy points and cut the rank a target
+// needs by 4-8%).  For l = 0 .. k-1:
+//   1. add component l back: R <- R + d_l u_l v_l^T (one fp32 add or
+//      subtract per touched entry);
+//   2. the old pattern, rescaled on this residual: p_o = u_l^T R W v_l,
+//      gain g_o = p_o^2 / (|u_l|^2 v_l^T W v_l), scale p_o / (|u_l|^2 v_l^T W v_l);
+//   3. the refit: `iters` ALS rounds from v = v_l, gain g_n and scale as in
+//      the greedy pass;
+//   4. the refit replaces the old pattern only if g_n > g_o; if the larger
+//      gain is below the best single entry's w_j R_ij^2, that entry is taken
+//      instead (Prop. 2);
+//   5. deflate with the choice and store it as component l.
+// Since the old pattern with its re-solved scale removes at least what d_l
+// did, no step raises |R|_W^2 (up to fp32 rounding of the updates).
+// step_flags[l]: bit 0 = single entry, bit 1 = old pattern kept.  Returns the
+// number of single-entry steps.
+int64_t orc_refine_sweep(float* R, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                         const float* w, int flags, int8_t* U, int8_t* V, float* D,
+                         uint8_t* step_flags) {
+  const int stat = flags & 1, naive = (flags >> 1) & 1;
+  std::vector<double> y(m), z(n);
+  std::vector<int8_t> u(m), v(n);
+  int64_t nsingle = 0;
+  for (int64_t l = 0; l < k; ++l) {
+    int8_t* Ul = U + l * m;
+    int8_t* Vl = V + l * n;
+    orc_deflate(R, m, n, Ul, Vl, -D[l]);  // add back
+    double p_old = 0.0, vw_old = 0.0;
+    int64_t nu_old = 0;
+    for (int64_t i = 0; i < m; ++i) {
+      if (!Ul[i]) continue;
+      ++nu_old;
+      for (int64_t j = 0; j < n; ++j)
+        if (Vl[j]) p_old += (double)Ul[i] * (double)R[i * n + j] * wt(w, j) * (double)Vl[j];
+    }
+    for (int64_t j = 0; j < n; ++j)
+      if (Vl[j]) vw_old += wt(w, j);
+    const double den_old = (double)nu_old * vw_old;
+    const double g_old = den_old > 0.0 ? p_old * p_old / den_old : 0.0;
+    std::memcpy(v.data(), Vl, n);
+    for (int t = 0; t < iters; ++t) {
+      orc_u_step2(R, m, n, v.data(), w, tau, stat, y.data(), u.data());
+      orc_v_step2(R, m, n, u.data(), w, tau, stat, naive, z.data(), v.data());
+    }
+    double sc[6];
+    orc_scale(z.data(), u.data(), v.data(), m, n, w, sc);
+    double M = 0.0;
+    const int64_t flat = orc_entry_max(R, m, n, w, &M);
+    uint8_t fl = 0;
+    float d;
+    const double g_best = sc[5] > g_old ? sc[5] : g_old;
+    if (g_best < M) {  // the best single entry beats both patterns
+      for (int64_t i = 0; i < m; ++i) u[i] = 0;
+      for (int64_t j = 0; j < n; ++j) v[j] = 0;
+      u[flat / n] = 1;
+      v[flat % n] = 1;
+      d = R[flat];
+      fl = 1;
+      ++nsingle;
+    } else if (sc[5] > g_old) {
+      d = (float)sc[4];
+    } else {
+      std::memcpy(u.data(), Ul, m);
+      std::memcpy(v.data(), Vl, n);
+      d = den_old > 0.0 ? (float)(p_old / den_old) : 0.0f;
+      fl = 2;
+    }
+    orc_deflate(R, m, n, u.data(), v.data(), d);
+    std::memcpy(Ul, u.data(), m);
+    std::memcpy(Vl, v.data(), n);
+    D[l] = d;
+    step_flags[l] = fl;
+  }
+  return nsingle;
 }
 
 // Replays components [0, upto) onto A with the same fp32 deflation; the
@@ -316,6 +446,18 @@ void orc_reconstruct(const int8_t* U, const int8_t* V, const float* D, int64_t m
   }
 }
 
+// Per-matrix rank allocation to an energy target ([REV] "Results": mu is set
+// per matrix so that its energy matches a reference quantiser's, 1.97 .. 3.43
+// per [PITH] "Assumptions & free parameters").  Greedy deflation fixes
+// components in order, so a run at rank k contains every shorter run as its
+// prefix; the smallest rank reaching the target is the first c with
+// energy[c] >= target, plus one.  Returns 0 when no prefix reaches it.
+int64_t orc_rank_for_energy(const double* energy, int64_t k, double target) {
+  for (int64_t c = 0; c < k; ++c)
+    if (energy[c] >= target) return c + 1;
+  return 0;
+}
+
 // Indices of the b largest row energies, distinct, descending, lowest index
 // first on ties (block-ALS initialisation).
 void orc_top_rows(const double* rho, int64_t m, int64_t b, int64_t* rows) {
@@ -331,8 +473,9 @@ void orc_top_rows(const double* rho, int64_t m, int64_t b, int64_t* rows) {
 // thresholded with its own rms over the m rows.  V and U are column-major
 // per component: V[l*n + j], U[l*m + i].  targets (m x bb, row-major, may be
 // NULL) receives the target, thr (bb, may be NULL) the thresholds.
-void orc_block_u_step(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* V,
-                      const float* w, double tau, int8_t* U, double* targets, double* thr) {
+void orc_block_u_step2(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* V,
+                       const float* w, double tau, int stat, int8_t* U, double* targets,
+                       double* thr) {
   std::vector<double> G(bb * bb);
   for (int64_t l = 0; l < bb; ++l)
     for (int64_t l2 = 0; l2 < bb; ++l2) {
@@ -353,16 +496,24 @@ void orc_block_u_step(const float* R, int64_t m, int64_t n, int64_t bb, const in
     }
   chol_solve(G, bb, Pt, m);
   for (int64_t l = 0; l < bb; ++l) {
-    const double t = orc_ternarize(&Pt[l * m], m, tau, U + l * m);
+    const double t = orc_ternarize2(&Pt[l * m], m, tau, stat, U + l * m);
     if (thr) thr[l] = t;
     if (targets)
       for (int64_t i = 0; i < m; ++i) targets[i * bb + l] = Pt[l * m + i];
   }
 }
 
-// Block-ALS V half-step (Eq. 3): V = T_col(((U^T U + eps I)^-1 U^T R)^T).
-void orc_block_v_step(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* U,
-                      double tau, int8_t* V, double* targets, double* thr) {
+void orc_block_u_step(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* V,
+                      const float* w, double tau, int8_t* U, double* targets, double* thr) {
+  orc_block_u_step2(R, m, n, bb, V, w, tau, 0, U, targets, thr);
+}
+
+// Block-ALS V half-step (Eq. 3): V = T_col(((U^T U + eps I)^-1 U^T R)^T); the
+// naive weighted V-step thresholds each column of W times that target.
+// targets (n x bb) receives the thresholded values (weighted when naive).
+void orc_block_v_step2(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* U,
+                       const float* w, double tau, int stat, int naive, int8_t* V,
+                       double* targets, double* thr) {
   std::vector<double> G(bb * bb);
   for (int64_t l = 0; l < bb; ++l)
     for (int64_t l2 = 0; l2 < bb; ++l2) {
@@ -380,12 +531,20 @@ void orc_block_v_step(const float* R, int64_t m, int64_t n, int64_t bb, const in
       for (int64_t j = 0; j < n; ++j) Q[l * n + j] += (double)ui * (double)R[i * n + j];
     }
   chol_solve(G, bb, Q, n);
+  if (naive && w)
+    for (int64_t l = 0; l < bb; ++l)
+      for (int64_t j = 0; j < n; ++j) Q[l * n + j] *= (double)w[j];
   for (int64_t l = 0; l < bb; ++l) {
-    const double t = orc_ternarize(&Q[l * n], n, tau, V + l * n);
+    const double t = orc_ternarize2(&Q[l * n], n, tau, stat, V + l * n);
     if (thr) thr[l] = t;
     if (targets)
       for (int64_t j = 0; j < n; ++j) targets[j * bb + l] = Q[l * n + j];
   }
+}
+
+void orc_block_v_step(const float* R, int64_t m, int64_t n, int64_t bb, const int8_t* U,
+                      double tau, int8_t* V, double* targets, double* thr) {
+  orc_block_v_step2(R, m, n, bb, U, nullptr, tau, 0, 0, V, targets, thr);
 }
 
 // Joint block scales: (G + eps I) D = r with G = (U^T U) o (V^T W V) and
@@ -432,14 +591,20 @@ void orc_block_scales(const float* R, int64_t m, int64_t n, int64_t bb, const in
   }
 }
 
-// Starting V of a block: column l = T_tau(R[rows[l], :]) (each row's own rms).
-void orc_block_init(const float* R, int64_t m, int64_t n, int64_t bb, const int64_t* rows,
-                    double tau, int8_t* V) {
+// Starting V of a block: column l = T_tau(R[rows[l], :]) (each row's own
+// statistic).
+void orc_block_init2(const float* R, int64_t m, int64_t n, int64_t bb, const int64_t* rows,
+                     double tau, int stat, int8_t* V) {
   std::vector<double> row(n);
   for (int64_t l = 0; l < bb; ++l) {
     for (int64_t j = 0; j < n; ++j) row[j] = (double)R[rows[l] * n + j];
-    orc_ternarize(row.data(), n, tau, V + l * n);
+    orc_ternarize2(row.data(), n, tau, stat, V + l * n);
   }
+}
+
+void orc_block_init(const float* R, int64_t m, int64_t n, int64_t bb, const int64_t* rows,
+                    double tau, int8_t* V) {
+  orc_block_init2(R, m, n, bb, rows, tau, 0, V);
 }
 
 // Block-ALS with decorrelated least-squares targets (paper Sec. 2.4, Eq. 3 per
@@ -448,9 +613,10 @@ void orc_block_init(const float* R, int64_t m, int64_t n, int64_t bb, const int6
 // rounds of the U and V half-steps above, joint scales, then bb ordered
 // rank-1 deflations.  Energy per component from the closed form
 // |R|^2 - 2 sum d_l r_l + sum d_l d_l' G_ll' over the block prefix.
-void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
-                         const float* w, int64_t b, int8_t* U, int8_t* V, float* D,
-                         double* energy, int64_t* init_row) {
+void orc_decompose_block2(const float* A, int64_t m, int64_t n, int64_t k, double tau,
+                          int iters, const float* w, int flags, int64_t b, int8_t* U, int8_t* V,
+                          float* D, double* energy, int64_t* init_row) {
+  const int stat = flags & 1, naive = (flags >> 1) & 1;
   std::vector<float> R(A, A + m * n);
   const double E0 = orc_sumsq(A, m, n, w);
   std::vector<double> rho(m);
@@ -461,10 +627,11 @@ void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double
     orc_top_rows(rho.data(), m, bb, rows.data());
     for (int64_t l = 0; l < bb; ++l) init_row[c0 + l] = rows[l];
     std::vector<int8_t> Ub(bb * m, 0), Vb(bb * n, 0);
-    orc_block_init(R.data(), m, n, bb, rows.data(), tau, Vb.data());
+    orc_block_init2(R.data(), m, n, bb, rows.data(), tau, stat, Vb.data());
     for (int t = 0; t < iters; ++t) {
-      orc_block_u_step(R.data(), m, n, bb, Vb.data(), w, tau, Ub.data(), nullptr, nullptr);
-      orc_block_v_step(R.data(), m, n, bb, Ub.data(), tau, Vb.data(), nullptr, nullptr);
+      orc_block_u_step2(R.data(), m, n, bb, Vb.data(), w, tau, stat, Ub.data(), nullptr, nullptr);
+      orc_block_v_step2(R.data(), m, n, bb, Ub.data(), w, tau, stat, naive, Vb.data(), nullptr,
+                        nullptr);
     }
     std::vector<double> dsol(bb), Graw(bb * bb), r(bb);
     orc_block_scales(R.data(), m, n, bb, Ub.data(), Vb.data(), w, dsol.data(), Graw.data(),
@@ -485,6 +652,12 @@ void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double
       energy[c0 + l] = E0 > 0.0 ? 1.0 - e / E0 : 1.0;
     }
   }
+}
+
+void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double tau, int iters,
+                         const float* w, int64_t b, int8_t* U, int8_t* V, float* D,
+                         double* energy, int64_t* init_row) {
+  orc_decompose_block2(A, m, n, k, tau, iters, w, 0, b, U, V, D, energy, init_row);
 }
 
 }  // extern "C"

@@ -31,6 +31,31 @@ def lib():
         L = ctypes.CDLL(_build.build())
         L.orc_ternarize.argtypes = [_D, _i64, ctypes.c_double, _I8]
         L.orc_ternarize.restype = ctypes.c_double
+        L.orc_ternarize2.argtypes = [_D, _i64, ctypes.c_double, ctypes.c_int, _I8]
+        L.orc_ternarize2.restype = ctypes.c_double
+        L.orc_u_step2.argtypes = [_F, _i64, _i64, _I8, _F, ctypes.c_double, ctypes.c_int, _D, _I8]
+        L.orc_u_step2.restype = ctypes.c_double
+        L.orc_v_step2.argtypes = [_F, _i64, _i64, _I8, _F, ctypes.c_double, ctypes.c_int,
+                                  ctypes.c_int, _D, _I8]
+        L.orc_v_step2.restype = ctypes.c_double
+        L.orc_decompose_seq2.argtypes = [_F, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _F,
+                                         ctypes.c_int, ctypes.c_int, _I8, _I8, _F, _D, _I64, _U8,
+                                         _D, _U8]
+        L.orc_decompose_seq2.restype = _i64
+        L.orc_refine_sweep.argtypes = [_F, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _F,
+                                       ctypes.c_int, _I8, _I8, _F, _U8]
+        L.orc_refine_sweep.restype = _i64
+        L.orc_block_u_step2.argtypes = [_F, _i64, _i64, _i64, _I8, _F, ctypes.c_double,
+                                        ctypes.c_int, _I8, _D, _D]
+        L.orc_block_u_step2.restype = None
+        L.orc_block_v_step2.argtypes = [_F, _i64, _i64, _i64, _I8, _F, ctypes.c_double,
+                                        ctypes.c_int, ctypes.c_int, _I8, _D, _D]
+        L.orc_block_v_step2.restype = None
+        L.orc_block_init2.argtypes = [_F, _i64, _i64, _i64, _I64, ctypes.c_double, ctypes.c_int, _I8]
+        L.orc_block_init2.restype = None
+        L.orc_decompose_block2.argtypes = [_F, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _F,
+                                           ctypes.c_int, _i64, _I8, _I8, _F, _D, _I64]
+        L.orc_decompose_block2.restype = None
         L.orc_u_step.argtypes = [_F, _i64, _i64, _I8, _F, ctypes.c_double, _D, _I8]
         L.orc_u_step.restype = ctypes.c_double
         L.orc_v_step.argtypes = [_F, _i64, _i64, _I8, ctypes.c_double, _D, _I8]
@@ -54,6 +79,8 @@ def lib():
         L.orc_replay_range.restype = None
         L.orc_reconstruct.argtypes = [_I8, _I8, _F, _i64, _i64, _i64, _D]
         L.orc_reconstruct.restype = None
+        L.orc_rank_for_energy.argtypes = [_D, _i64, ctypes.c_double]
+        L.orc_rank_for_energy.restype = _i64
         L.orc_top_rows.argtypes = [_D, _i64, _i64, _I64]
         L.orc_top_rows.restype = None
         L.orc_block_u_step.argtypes = [_F, _i64, _i64, _i64, _I8, _F, ctypes.c_double, _I8, _D, _D]
@@ -82,28 +109,49 @@ def _f32(a):
     return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
 
 
-def ternarize(x: np.ndarray, tau: float):
+# variant flags (same bits as the library's): threshold statistic mean |x|,
+# naive weighted V-step
+MEAN_ABS = 1
+NAIVE_VSTEP = 2
+
+
+def ternarize(x: np.ndarray, tau: float, stat: int = 0):
+    """T_tau with the rms (stat 0) or mean-|x| (stat 1) statistic."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     out = np.empty(x.shape[0], np.int8)
-    thr = lib().orc_ternarize(_p(x, _D), x.shape[0], tau, _p(out, _I8))
+    if stat == 0:
+        thr = lib().orc_ternarize(_p(x, _D), x.shape[0], tau, _p(out, _I8))
+    else:
+        thr = lib().orc_ternarize2(_p(x, _D), x.shape[0], tau, stat, _p(out, _I8))
     return out, thr
 
 
-def u_step(R: np.ndarray, v: np.ndarray, tau: float, w=None):
+def u_step(R: np.ndarray, v: np.ndarray, tau: float, w=None, stat: int = 0):
     R = _f32(R); w = _f32(w)
     m, n = R.shape
     v = np.ascontiguousarray(v, np.int8)
     y = np.empty(m); u = np.empty(m, np.int8)
-    thr = lib().orc_u_step(_p(R, _F), m, n, _p(v, _I8), _p(w, _F), tau, _p(y, _D), _p(u, _I8))
+    if stat == 0:
+        thr = lib().orc_u_step(_p(R, _F), m, n, _p(v, _I8), _p(w, _F), tau, _p(y, _D), _p(u, _I8))
+    else:
+        thr = lib().orc_u_step2(_p(R, _F), m, n, _p(v, _I8), _p(w, _F), tau, stat, _p(y, _D),
+                                _p(u, _I8))
     return u, y, thr
 
 
-def v_step(R: np.ndarray, u: np.ndarray, tau: float):
+def v_step(R: np.ndarray, u: np.ndarray, tau: float, w=None, stat: int = 0, naive: bool = False):
+    """v = T_tau(R^T u), or T_tau(w o R^T u) for the naive weighted V-step;
+    returns (v, z = R^T u unweighted, threshold)."""
     R = _f32(R)
     m, n = R.shape
     u = np.ascontiguousarray(u, np.int8)
     z = np.empty(n); v = np.empty(n, np.int8)
-    thr = lib().orc_v_step(_p(R, _F), m, n, _p(u, _I8), tau, _p(z, _D), _p(v, _I8))
+    if stat == 0 and not naive:
+        thr = lib().orc_v_step(_p(R, _F), m, n, _p(u, _I8), tau, _p(z, _D), _p(v, _I8))
+    else:
+        w = _f32(w)
+        thr = lib().orc_v_step2(_p(R, _F), m, n, _p(u, _I8), _p(w, _F), tau, stat, int(naive),
+                                _p(z, _D), _p(v, _I8))
     return v, z, thr
 
 
@@ -161,29 +209,59 @@ class Decomposition:
     U: np.ndarray         # k x m int8 (B^T)
     V: np.ndarray         # k x n int8 (C)
     D: np.ndarray         # k fp32
-    energy: np.ndarray    # k fp64
+    energy: np.ndarray    # k fp64 (the greedy pass)
     init_row: np.ndarray  # k int64
     fallback: np.ndarray  # k uint8 (sequential mode only)
     n_fallback: int
+    sweep_energy: np.ndarray = None  # [sweeps] fp64: energy after each refinement sweep
+    sweep_flags: np.ndarray = None   # [sweeps, k] uint8: bit 0 single entry, bit 1 old kept
 
 
 def decompose(A, k: int, tau: float, iters: int, w=None, block: int = 1,
-              block_path: bool = False) -> Decomposition:
-    """Free-running decomposition; block > 1 (or block_path) runs block-ALS."""
+              block_path: bool = False, flags: int = 0, sweeps: int = 0) -> Decomposition:
+    """Free-running decomposition; block > 1 (or block_path) runs block-ALS.
+    flags: MEAN_ABS | NAIVE_VSTEP; sweeps: refinement sweeps (sequential)."""
     A = _f32(A); w = _f32(w)
     m, n = A.shape
     U = np.zeros((k, m), np.int8); V = np.zeros((k, n), np.int8)
     D = np.zeros(k, np.float32); E = np.zeros(k); rows = np.zeros(k, np.int64)
     fb = np.zeros(k, np.uint8)
+    se = np.zeros(max(sweeps, 1)); sf = np.zeros((max(sweeps, 1), k), np.uint8)
     if block <= 1 and not block_path:
-        nfb = lib().orc_decompose_seq(_p(A, _F), m, n, k, tau, iters, _p(w, _F), _p(U, _I8),
-                                      _p(V, _I8), _p(D, _F), _p(E, _D), _p(rows, _I64),
-                                      _p(fb, _U8))
+        if flags == 0 and sweeps == 0:
+            nfb = lib().orc_decompose_seq(_p(A, _F), m, n, k, tau, iters, _p(w, _F), _p(U, _I8),
+                                          _p(V, _I8), _p(D, _F), _p(E, _D), _p(rows, _I64),
+                                          _p(fb, _U8))
+        else:
+            nfb = lib().orc_decompose_seq2(_p(A, _F), m, n, k, tau, iters, _p(w, _F), flags,
+                                           sweeps, _p(U, _I8), _p(V, _I8), _p(D, _F), _p(E, _D),
+                                           _p(rows, _I64), _p(fb, _U8), _p(se, _D), _p(sf, _U8))
     else:
-        lib().orc_decompose_block(_p(A, _F), m, n, k, tau, iters, _p(w, _F), block, _p(U, _I8),
-                                  _p(V, _I8), _p(D, _F), _p(E, _D), _p(rows, _I64))
+        if flags == 0:
+            lib().orc_decompose_block(_p(A, _F), m, n, k, tau, iters, _p(w, _F), block,
+                                      _p(U, _I8), _p(V, _I8), _p(D, _F), _p(E, _D),
+                                      _p(rows, _I64))
+        else:
+            lib().orc_decompose_block2(_p(A, _F), m, n, k, tau, iters, _p(w, _F), flags, block,
+                                       _p(U, _I8), _p(V, _I8), _p(D, _F), _p(E, _D),
+                                       _p(rows, _I64))
         nfb = 0
-    return Decomposition(U, V, D, E, rows, fb, int(nfb))
+    return Decomposition(U, V, D, E, rows, fb, int(nfb), se[:sweeps], sf[:sweeps])
+
+
+def refine_sweep(R, U, V, D, tau: float, iters: int, w=None, flags: int = 0):
+    """One refinement sweep on copies: returns (R, U, V, D, step_flags)."""
+    R = np.array(R, dtype=np.float32, order="C", copy=True)
+    U = np.array(U, dtype=np.int8, order="C", copy=True)
+    V = np.array(V, dtype=np.int8, order="C", copy=True)
+    D = np.array(D, dtype=np.float32, order="C", copy=True)
+    w = _f32(w)
+    m, n = R.shape
+    k = D.shape[0]
+    fl = np.zeros(k, np.uint8)
+    lib().orc_refine_sweep(_p(R, _F), m, n, k, tau, iters, _p(w, _F), flags, _p(U, _I8),
+                           _p(V, _I8), _p(D, _F), _p(fl, _U8))
+    return R, U, V, D, fl
 
 
 def replay(A, U, V, D, upto: int) -> np.ndarray:
@@ -213,6 +291,12 @@ def reconstruct(U, V, D, m: int, n: int) -> np.ndarray:
     return out
 
 
+def rank_for_energy(energy, target: float) -> int:
+    """Smallest rank r whose prefix reaches the energy target (0: none)."""
+    e = np.ascontiguousarray(energy, np.float64)
+    return int(lib().orc_rank_for_energy(_p(e, _D), e.shape[0], target))
+
+
 def top_rows(rho, b: int):
     rho = np.ascontiguousarray(rho, np.float64)
     rows = np.empty(b, np.int64)
@@ -222,35 +306,37 @@ def top_rows(rho, b: int):
 
 # --- block-ALS half-steps (component-major codes: U[l, i], V[l, j]) ---------
 
-def block_init(R, rows, tau):
+def block_init(R, rows, tau, stat: int = 0):
     R = _f32(R)
     m, n = R.shape
     rows = np.ascontiguousarray(rows, np.int64)
     V = np.zeros((rows.shape[0], n), np.int8)
-    lib().orc_block_init(_p(R, _F), m, n, rows.shape[0], _p(rows, _I64), tau, _p(V, _I8))
+    lib().orc_block_init2(_p(R, _F), m, n, rows.shape[0], _p(rows, _I64), tau, stat, _p(V, _I8))
     return V
 
 
-def block_u_step(R, V, tau, w=None):
+def block_u_step(R, V, tau, w=None, stat: int = 0):
     R = _f32(R); w = _f32(w)
     m, n = R.shape
     V = np.ascontiguousarray(V, np.int8)
     bb = V.shape[0]
     U = np.zeros((bb, m), np.int8)
     T = np.zeros((m, bb)); thr = np.zeros(bb)
-    lib().orc_block_u_step(_p(R, _F), m, n, bb, _p(V, _I8), _p(w, _F), tau, _p(U, _I8), _p(T, _D),
-                           _p(thr, _D))
+    lib().orc_block_u_step2(_p(R, _F), m, n, bb, _p(V, _I8), _p(w, _F), tau, stat, _p(U, _I8),
+                            _p(T, _D), _p(thr, _D))
     return U, T, thr
 
 
-def block_v_step(R, U, tau):
-    R = _f32(R)
+def block_v_step(R, U, tau, w=None, stat: int = 0, naive: bool = False):
+    """V half-step; T is the thresholded target (times w when naive)."""
+    R = _f32(R); w = _f32(w)
     m, n = R.shape
     U = np.ascontiguousarray(U, np.int8)
     bb = U.shape[0]
     V = np.zeros((bb, n), np.int8)
     T = np.zeros((n, bb)); thr = np.zeros(bb)
-    lib().orc_block_v_step(_p(R, _F), m, n, bb, _p(U, _I8), tau, _p(V, _I8), _p(T, _D), _p(thr, _D))
+    lib().orc_block_v_step2(_p(R, _F), m, n, bb, _p(U, _I8), _p(w, _F), tau, stat, int(naive),
+                            _p(V, _I8), _p(T, _D), _p(thr, _D))
     return V, T, thr
 
 

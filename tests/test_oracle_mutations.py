@@ -38,6 +38,18 @@ MUTATIONS = [
     ("block_u_target_unweighted", "s += (double)R[i * n + j] * wt(w, j) * V[l * n + j];",
      "s += (double)R[i * n + j] * V[l * n + j];"),
     ("safeguard_score_drops_weight", "float s = sq * w[j];", "float s = sq;"),
+    ("mean_abs_statistic_ignored", "s += stat == 1 ? std::fabs(x[j]) : x[j] * x[j];",
+     "s += x[j] * x[j];"),
+    ("naive_vstep_drops_weight", "wz[j] = (double)w[j] * z[j];", "wz[j] = z[j];"),
+    ("block_naive_drops_weight", "for (int64_t j = 0; j < n; ++j) Q[l * n + j] *= (double)w[j];",
+     "for (int64_t j = 0; j < n; ++j) Q[l * n + j] *= 1.0;"),
+    ("sweep_addback_sign", "orc_deflate(R, m, n, Ul, Vl, -D[l]);  // add back",
+     "orc_deflate(R, m, n, Ul, Vl, D[l]);  // add back"),
+    ("sweep_choice_flipped", "} else if (sc[5] > g_old) {", "} else if (sc[5] < g_old) {"),
+    ("sweep_old_scale_not_resolved", "d = den_old > 0.0 ? (float)(p_old / den_old) : 0.0f;",
+     "d = D[l];"),
+    ("sweep_single_entry_ignores_old", "const double g_best = sc[5] > g_old ? sc[5] : g_old;",
+     "const double g_best = sc[5];"),
 ]
 
 PIN_TESTS = [
@@ -60,6 +72,12 @@ PIN_TESTS = [
     pins.test_block_energy_matches_replay,
     pins.test_exact_recovery_of_ternary_rank1,
     pins.test_exact_recovery_of_two_disjoint_components,
+    pins.test_ternarize_mean_abs_hand_computed,
+    pins.test_naive_vstep_against_numpy,
+    lambda o: pins.test_block_variant_targets(o, True),
+    lambda o: pins.test_sweep_steps_match_a_replay_by_hand(o, False),
+    lambda o: pins.test_sweep_steps_match_a_replay_by_hand(o, True),
+    pins.test_sweeps_never_raise_the_residual,
 ]
 
 
