@@ -9,8 +9,10 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libexternd.so")
+# (-static-global-template-stub=false: the sequential kernel template is
+# instantiated in its own units and launched from seq_als.cu)
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-              "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
+              "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-static-global-template-stub=false"]
 
 
 def sources():
@@ -32,14 +34,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "nvcc")
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *NVCC_FLAGS, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # the translation units are independent: compile them side by side
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as ex:
+        for r in list(ex.map(lambda c: subprocess.run(c, check=True), cmds)):
+            pass
     tmp = LIB + ".tmp"
     subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", *objs, "-o", tmp,
                     "-lcudart"], check=True)
@@ -53,7 +60,7 @@ if __name__ == "__main__":
 
 # the source files each profiled kernel is built from
 KERNEL_SOURCES = {
-    "seq_als_kernel": ("seq_als.cu", "common.cuh"),
+    "seq_als_kernel": ("seq_als.cu", "seq_kernel.cuh", "seq_inst_smem_plain.cu", "common.cuh"),
     "contract_tma_kernel": ("umma_contract.cu", "umma_layout.cuh", "common.cuh"),
 }
 

@@ -1,0 +1,8 @@
+// Instantiates the sequential kernel for tiles partly in global memory, with the
+// threshold variants and refinement sweeps (one unit per case, so the
+// instantiations compile side by side).
+#include "seq_kernel.cuh"
+
+namespace externd {
+EXTERND_SEQ_KERNELS(true, true, )
+}  // namespace externd
