@@ -30,8 +30,9 @@ int64_t externd_rank(int64_t m, int64_t n, float mu) {
 }
 
 int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
-                             const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
-                             float* D, double* energy_trace, int64_t ntrace,
+                             const float* w, int block, unsigned flags, int sweeps,
+                             uint32_t* packed_B, uint32_t* packed_C, float* D,
+                             double* energy_trace, double* sweep_energy, int64_t ntrace,
                              const int64_t* trace_comp, uint32_t* trace_bits, int32_t* trace_row,
                              uint8_t* trace_flags, int64_t* stats, int64_t wait_budget,
                              externd_stream_t stream) {
@@ -45,6 +46,11 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
   if (!(tau >= 0.0f) || !std::isfinite(tau)) return EXTERND_ERR_INVALID_ARG;
   if (iters < 1 || iters > 1000) return EXTERND_ERR_INVALID_ARG;
   if (block < 1 || block > 64 || block > k || block > (m < n ? m : n)) return EXTERND_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)(EXTERND_TSTAT_MEAN_ABS | EXTERND_VSTEP_NAIVE)) return EXTERND_ERR_INVALID_ARG;
+  if (sweeps < 0 || sweeps > EXTERND_MAX_SWEEPS || (sweeps > 0 && block != 1))
+    return EXTERND_ERR_INVALID_ARG;
+  if (sweeps > 0 && (!sweep_energy || ((uintptr_t)sweep_energy & 7u))) return EXTERND_ERR_INVALID_ARG;
+  if (k * (1 + (int64_t)sweeps) > 2147483647LL) return EXTERND_ERR_INVALID_ARG;
   if (ntrace < 0 || wait_budget < 0) return EXTERND_ERR_INVALID_ARG;
   if (ntrace > 0 && (!trace_comp || !trace_bits || !trace_row || !trace_flags || block != 1))
     return EXTERND_ERR_INVALID_ARG;
@@ -56,17 +62,20 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
     h.packed_B = packed_B; h.packed_C = packed_C; h.D = D; h.energy = energy_trace;
     h.ntrace = ntrace; h.trace_comp = trace_comp; h.trace_bits = trace_bits;
     h.trace_row = trace_row; h.trace_flags = trace_flags; h.stats = stats;
-    h.wait_budget = wait_budget;
+    h.wait_budget = wait_budget; h.flags = flags; h.sweeps = sweeps;
+    h.sweep_energy = sweep_energy;
     return externd::seq_decompose(h, st);
   }
   externd::BlockHostArgs b = {};
   b.A = A; b.m = m; b.n = n; b.k = k; b.tau = tau; b.iters = iters; b.w = w; b.block = block;
   b.packed_B = packed_B; b.packed_C = packed_C; b.D = D; b.energy = energy_trace; b.stats = stats;
+  b.flags = flags;
   return externd::block_decompose(b, st);
 }
 
 int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float mu, float tau,
-                                   int iters, const float* w, int block, uint32_t* packed_B,
+                                   int iters, const float* w, int block, unsigned flags,
+                                   uint32_t* packed_B,
                                    uint32_t* packed_C, float* D, double* energy_trace,
                                    int64_t ntrace, const int64_t* trace_block, uint64_t* trace_uv,
                                    int32_t* trace_rows, externd_stream_t stream) {
@@ -83,19 +92,29 @@ int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float m
   if (!(tau >= 0.0f) || !std::isfinite(tau)) return EXTERND_ERR_INVALID_ARG;
   if (iters < 1 || iters > 1000) return EXTERND_ERR_INVALID_ARG;
   if (block > 64 || block > k || block > (m < n ? m : n)) return EXTERND_ERR_INVALID_ARG;
+  if (flags & ~(unsigned)(EXTERND_TSTAT_MEAN_ABS | EXTERND_VSTEP_NAIVE)) return EXTERND_ERR_INVALID_ARG;
   externd::BlockHostArgs b = {};
   b.A = A; b.m = m; b.n = n; b.k = k; b.tau = tau; b.iters = iters; b.w = w; b.block = block;
   b.packed_B = packed_B; b.packed_C = packed_C; b.D = D; b.energy = energy_trace;
   b.ntrace = ntrace; b.trace_block = trace_block; b.trace_uv = trace_uv; b.trace_rows = trace_rows;
+  b.flags = flags;
   return externd::block_decompose(b, (cudaStream_t)stream);
+}
+
+int externd_decompose_ex(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
+                         const float* w, int block, unsigned flags, int sweeps,
+                         uint32_t* packed_B, uint32_t* packed_C, float* D, double* energy_trace,
+                         double* sweep_energy, externd_stream_t stream) {
+  return externd_decompose_traced(A, m, n, mu, tau, iters, w, block, flags, sweeps, packed_B,
+                                  packed_C, D, energy_trace, sweep_energy, 0, nullptr, nullptr,
+                                  nullptr, nullptr, nullptr, 0, stream);
 }
 
 int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
                       const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
                       float* D, double* energy_trace, externd_stream_t stream) {
-  return externd_decompose_traced(A, m, n, mu, tau, iters, w, block, packed_B, packed_C, D,
-                                  energy_trace, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0,
-                                  stream);
+  return externd_decompose_ex(A, m, n, mu, tau, iters, w, block, 0u, 0, packed_B, packed_C, D,
+                              energy_trace, nullptr, stream);
 }
 
 int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, const float* D,

@@ -269,15 +269,17 @@ __global__ void __launch_bounds__(1024) select_rows_kernel(const double* __restr
 }
 
 // ---- starting V: column l = T_tau(R[rows[l], :]) ----------------------------
+// (stat 0: threshold tau * rms of the row; stat 1: tau * mean |x|)
 __global__ void vinit_kernel(const float* __restrict__ R, int n, const int* __restrict__ rows,
-                             double tau, u64* __restrict__ Vm, u64* __restrict__ Vs) {
+                             double tau, int stat, u64* __restrict__ Vm, u64* __restrict__ Vs) {
   __shared__ double sh[32];
   const int l = blockIdx.x;
   const float* row = R + (size_t)rows[l] * n;
   double s = 0.0;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) s += (double)row[j] * (double)row[j];
+  for (int j = threadIdx.x; j < n; j += blockDim.x)
+    s += stat ? fabs((double)row[j]) : (double)row[j] * (double)row[j];
   s = block_sum_d(s, sh);
-  const double thr = tau * sqrt(s / (double)n);
+  const double thr = stat ? tau * (s / (double)n) : tau * sqrt(s / (double)n);
   for (int j = threadIdx.x; j < n; j += blockDim.x) {
     const float x = row[j];
     if (fabs((double)x) > thr) {
@@ -466,111 +468,6 @@ __global__ void __launch_bounds__(256, 1) inv_kernel(const double* __restrict__ 
   }
 }
 
-// ---- contractions on CUDA cores ---------------------------------------------
-// P partials: Pp[split][i][l] = sum_{j in split} R_ij w_j s_jl   (64 x 64 tile)
-constexpr int kTile = 64, kKc = 32;
-__global__ void __launch_bounds__(256) rv_kernel(const float* __restrict__ R, int m, int n,
-                                                 const u64* __restrict__ Vm,
-                                                 const u64* __restrict__ Vs,
-                                                 const float* __restrict__ w, int bb, int klen,
-                                                 float* __restrict__ Pp) {
-  __shared__ __align__(16) float As[kKc][kTile + 4];
-  __shared__ __align__(16) float Bs[kKc][kTile];
-  const int i0 = blockIdx.x * kTile, split = blockIdx.y;
-  const int j0 = split * klen, j1 = min(n, j0 + klen);
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int jc = j0; jc < j1; jc += kKc) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < kTile * kKc; e += 256) {
-      const int r = e / kKc, kk = e - r * kKc;
-      const int i = i0 + r, j = jc + kk;
-      As[kk][r] = (i < m && j < j1) ? R[(size_t)i * n + j] : 0.f;
-    }
-    for (int e = threadIdx.x; e < kKc * kTile; e += 256) {
-      const int kk = e / kTile, l = e - kk * kTile;
-      const int j = jc + kk;
-      float v = 0.f;
-      if (j < j1 && l < bb) {
-        const u64 mm = Vm[j];
-        if ((mm >> l) & 1ull) v = (((Vs[j] >> l) & 1ull) ? -1.f : 1.f) * (w ? w[j] : 1.f);
-      }
-      Bs[kk][l] = v;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kKc; ++kk) {
-      const float4 a = *(const float4*)&As[kk][ty * 4];
-      const float4 b = *(const float4*)&Bs[kk][tx * 4];
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-  }
-  float* out = Pp + (size_t)split * m * bb;
-  for (int r = 0; r < 4; ++r) {
-    const int i = i0 + ty * 4 + r;
-    if (i >= m) continue;
-    for (int c = 0; c < 4; ++c) {
-      const int l = tx * 4 + c;
-      if (l < bb) out[(size_t)i * bb + l] = acc[r][c];
-    }
-  }
-}
-
-// Q partials: Qp[split][j][l] = sum_{i in split} R_ij s_il   (64 x 64 tile)
-__global__ void __launch_bounds__(256) rtu_kernel(const float* __restrict__ R, int m, int n,
-                                                  const u64* __restrict__ Um,
-                                                  const u64* __restrict__ Us, int bb, int klen,
-                                                  float* __restrict__ Qp) {
-  __shared__ __align__(16) float As[kKc][kTile];
-  __shared__ __align__(16) float Bs[kKc][kTile];
-  const int j0c = blockIdx.x * kTile, split = blockIdx.y;
-  const int r0 = split * klen, r1 = min(m, r0 + klen);
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4] = {};
-  for (int ic = r0; ic < r1; ic += kKc) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < kKc * kTile; e += 256) {
-      const int kk = e / kTile, c = e - kk * kTile;
-      const int i = ic + kk, j = j0c + c;
-      As[kk][c] = (i < r1 && j < n) ? R[(size_t)i * n + j] : 0.f;
-    }
-    for (int e = threadIdx.x; e < kKc * kTile; e += 256) {
-      const int kk = e / kTile, l = e - kk * kTile;
-      const int i = ic + kk;
-      float v = 0.f;
-      if (i < r1 && l < bb) {
-        const u64 mm = Um[i];
-        if ((mm >> l) & 1ull) v = ((Us[i] >> l) & 1ull) ? -1.f : 1.f;
-      }
-      Bs[kk][l] = v;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kKc; ++kk) {
-      const float4 a = *(const float4*)&As[kk][ty * 4];
-      const float4 b = *(const float4*)&Bs[kk][tx * 4];
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
-    }
-  }
-  float* out = Qp + (size_t)split * n * bb;
-  for (int r = 0; r < 4; ++r) {
-    const int j = j0c + ty * 4 + r;
-    if (j >= n) continue;
-    for (int c = 0; c < 4; ++c) {
-      const int l = tx * 4 + c;
-      if (l < bb) out[(size_t)j * bb + l] = acc[r][c];
-    }
-  }
-}
-
 // ---- targets: T[x][l] = sum_l2 (sum_s Xp[s][x][l2]) S[l2][l] (fp64) ----------
 // 64 rows per CTA, two CTAs per SM (one wave for up to 2 x SMs x 64 rows).
 // The split-K partials are summed (split order, fp64) into a transposed tile
@@ -580,8 +477,11 @@ __global__ void __launch_bounds__(256) rtu_kernel(const float* __restrict__ R, i
 // 4rg.., columns 4cg.. of T: 16 independent fp64 chains per thread.  Each CTA
 // writes its column sums of squares; the last CTA to finish (ticket counter)
 // sums those partials in CTA order and writes the column thresholds
-// thr[l] = tau * rms(T[:, l]), then rearms the counter.  With Xout set, the
-// split-summed X (rows x bb, fp64) is stored as well.
+// thr[l] = tau * rms(T[:, l]) (stat 0) or tau * mean |T[:, l]| (stat 1), then
+// rearms the counter.  With Xout set, the split-summed X (rows x bb, fp64) is
+// stored as well.  With wsc set, row x of T is scaled by wsc[x] before it is
+// stored and measured (the naive weighted V-step thresholds W times the
+// target).
 constexpr int kTgtRows2 = 64;  // rows per CTA of target_kernel
 constexpr int kMaxSplits = kMaxSegs;  // partials per output row (split-K or stream-K)
 constexpr int kXs = kTgtRows2 + 2;  // padded row of the transposed tile (16-byte aligned)
@@ -597,7 +497,8 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
                                                         unsigned* __restrict__ ticket,
                                                         double* __restrict__ thr,
                                                         double* __restrict__ Xout, int sk, int C,
-                                                        long long U, int G, int Sslots) {
+                                                        long long U, int G, int Sslots, int stat,
+                                                        const float* __restrict__ wsc) {
   extern __shared__ __align__(16) double tsh[];
   double* Ss = tsh;                                                 // [64][64]: S[l2][l]
   double* Xt = tsh + kMaxB * kMaxB;                                 // [64][kXs]
@@ -700,6 +601,11 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int x = x0 + 4 * rg + i;
+    if (x < rows && wsc) {
+      const double ws = (double)wsc[x];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] *= ws;
+    }
     if (x < rows) {
       if (bb == kMaxB) {
         *(double2*)(T + (size_t)x * bb + 4 * cg) = make_double2(acc[i][0], acc[i][1]);
@@ -710,7 +616,7 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
           if (4 * cg + j < bb) T[(size_t)x * bb + 4 * cg + j] = acc[i][j];
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) cs[j] += acc[i][j] * acc[i][j];
+      for (int j = 0; j < 4; ++j) cs[j] += stat ? fabs(acc[i][j]) : acc[i][j] * acc[i][j];
     }
   }
 #pragma unroll
@@ -750,7 +656,7 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
     __syncthreads();
     if (tid < bb) {
       const double t4 = ((part[0][tid] + part[1][tid]) + part[2][tid]) + part[3][tid];
-      thr[tid] = tau * sqrt(t4 / (double)rows);
+      thr[tid] = stat ? tau * (t4 / (double)rows) : tau * sqrt(t4 / (double)rows);
     }
   }
   if (tid == 0) *ticket = 0u;
@@ -758,7 +664,8 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
 constexpr size_t kTgtSmem = sizeof(double) * (kMaxB * kMaxB + kMaxB * kXs + 16 * kMaxB);
 // the target kernel instantiated for a split-count bound
 typedef void (*TargetFn)(const float*, int, int, int, const double*, double, double*, double*,
-                         unsigned*, double*, double*, int, int, long long, int, int);
+                         unsigned*, double*, double*, int, int, long long, int, int, int,
+                         const float*);
 inline TargetFn target_for(int splits) {
   if (splits <= 1) return target_kernel<1>;
   if (splits <= 2) return target_kernel<2>;
@@ -1067,12 +974,12 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
   int dev = 0, nsm = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  // Contractions run on the tensor cores (tcgen05, 128-row tiles); setting
-  // EXTERND_BLOCK_CUDA_CORES=1 selects the CUDA-core kernels (64-row tiles)
-  // instead, for comparison.
-  const char* cc = getenv("EXTERND_BLOCK_CUDA_CORES");
-  const bool tc = !(cc && cc[0] == '1');
-  const int tileR = tc ? 128 : kTile, kq = 32;
+  // contractions run on the tensor cores (tcgen05, 128-row tiles)
+  const int tileR = 128, kq = 32;
+  // threshold variants: the statistic of T_tau, and the weights the naive
+  // V-step scales its target by
+  const int stat = (h.flags & EXTERND_TSTAT_MEAN_ABS) ? 1 : 0;
+  const float* naive_w = (h.flags & EXTERND_VSTEP_NAIVE) ? h.w : nullptr;
   // split-K factors so each contraction has about two CTAs per SM
   const int tiles_m = (m + tileR - 1) / tileR, tiles_n = (n + tileR - 1) / tileR;
   // (at most two CTAs per SM in total, so a contraction runs in one wave)
@@ -1084,7 +991,7 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
   splitQ = (m + klenQ - 1) / klenQ;
   // the persistent TMA contraction (stream-K partials) whenever R's rows are
   // TMA-addressable; the workspace keeps R at a 256-byte aligned offset
-  const bool sk = tc && tc_contract_tma_ok(n);
+  const bool sk = tc_contract_tma_ok(n);
   TcPlan planP{}, planQ{};
   if (sk) {
     tc_contract_plan(m, n, nsm, &planP);
@@ -1149,8 +1056,8 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
   int* bad = (int*)(base + oBad);
   double* thr = (double*)(base + oThr);
   double* Qs = (double*)(base + oQs);
-  unsigned char* BopU = tc ? (unsigned char*)(base + oBopU) : nullptr;
-  unsigned char* BopV = tc ? (unsigned char*)(base + oBopV) : nullptr;
+  unsigned char* BopU = (unsigned char*)(base + oBopU);
+  unsigned char* BopV = (unsigned char*)(base + oBopV);
   float* wpad = (float*)(base + oWpad);
   unsigned* tick = (unsigned*)(base + oTick);
   const double tau = (double)h.tau;
@@ -1193,7 +1100,7 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
                                                   sel_smem > 0);
     cudaMemsetAsync(Vm, 0, sizeof(u64) * n, st);
     cudaMemsetAsync(Vs, 0, sizeof(u64) * n, st);
-    vinit_kernel<<<bb, 256, 0, st>>>(R, n, rows, tau, Vm, Vs);
+    vinit_kernel<<<bb, 256, 0, st>>>(R, n, rows, tau, stat, Vm, Vs);
     planes_kernel<<<(Wn * 32 + 255) / 256, 256, 0, st>>>(Vm, Vs, n, bb, pC, Wn, BopV);
     if (tr) {
       cudaMemcpyAsync(h.trace_rows + (size_t)tslot * b, rows, sizeof(int) * bb,
@@ -1208,28 +1115,22 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
       gram_kernel<<<gblocks, gthreads, 0, side>>>(pC, Wn, bb, h.w, GV);
       inv_kernel<<<1, 256, 0, side>>>(GV, bb, SV);
       cudaEventRecord(ev_join, side);
-      if (tc)
-        tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, sk ? &planP : nullptr, klenP, splitP,
-                       Pp, st);
-      else
-        rv_kernel<<<dim3(tiles_m, splitP), 256, 0, st>>>(R, m, n, Vm, Vs, h.w, bb, klenP, Pp);
+      tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, sk ? &planP : nullptr, klenP, splitP,
+                     Pp, st);
       cudaStreamWaitEvent(st, ev_join, 0);
       tgtP<<<tgtU, 256, kTgtSmem, st>>>(Pp, splitP, m, bb, SV, tau, T, Cs, tick, thr, nullptr, sk,
-                                         planP.C, planP.U, planP.G, planP.S);
+                                         planP.C, planP.U, planP.G, planP.S, stat, nullptr);
       tern_kernel<<<(Wm * 32 + 63) / 64, 64, 0, st>>>(T, m, bb, thr, Um, Us, pB, Wm, BopU);
       cudaEventRecord(ev_fork, st);
       cudaStreamWaitEvent(side, ev_fork, 0);
       gram_kernel<<<gblocks, gthreads, 0, side>>>(pB, Wm, bb, nullptr, GU);
       inv_kernel<<<1, 256, 0, side>>>(GU, bb, SU);
       cudaEventRecord(ev_join, side);
-      if (tc)
-        tc_contract_rtu(R, m, n, Um, Us, BopU, bb, sk ? &planQ : nullptr, klenQ, splitQ, Qp, st);
-      else
-        rtu_kernel<<<dim3(tiles_n, splitQ), 256, 0, st>>>(R, m, n, Um, Us, bb, klenQ, Qp);
+      tc_contract_rtu(R, m, n, Um, Us, BopU, bb, sk ? &planQ : nullptr, klenQ, splitQ, Qp, st);
       cudaStreamWaitEvent(st, ev_join, 0);
       tgtQ<<<tgtV, 256, kTgtSmem, st>>>(Qp, splitQ, n, bb, SU, tau, T, Cs, tick, thr,
                                          it == h.iters - 1 ? Qs : nullptr, sk, planQ.C, planQ.U,
-                                         planQ.G, planQ.S);
+                                         planQ.G, planQ.S, stat, naive_w);
       tern_kernel<<<(Wn * 32 + 63) / 64, 64, 0, st>>>(T, n, bb, thr, Vm, Vs, pC, Wn, BopV);
       if (tr) {
         u64* at = tr + 2 * (size_t)n + (size_t)it * 2 * ((size_t)m + n);
@@ -1261,13 +1162,12 @@ namespace {
 
 struct GraphKey {
   BlockHostArgs h;
-  int dev, cuda_cores, no_tma;
+  int dev, no_tma;
   bool operator==(const GraphKey& o) const {
     return h.A == o.h.A && h.m == o.h.m && h.n == o.h.n && h.k == o.h.k && h.tau == o.h.tau &&
            h.iters == o.h.iters && h.w == o.h.w && h.block == o.h.block &&
-           h.packed_B == o.h.packed_B && h.packed_C == o.h.packed_C && h.D == o.h.D &&
-           h.energy == o.h.energy && dev == o.dev && cuda_cores == o.cuda_cores &&
-           no_tma == o.no_tma;
+           h.flags == o.h.flags && h.packed_B == o.h.packed_B && h.packed_C == o.h.packed_C &&
+           h.D == o.h.D && h.energy == o.h.energy && dev == o.dev && no_tma == o.no_tma;
   }
 };
 
@@ -1370,8 +1270,7 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
     cudaGetLastError();
     return enqueue_direct(h, st);
   }
-  GraphKey key{h, 0, env_on("EXTERND_BLOCK_CUDA_CORES") ? 1 : 0,
-               getenv("EXTERND_CONTRACT_NO_TMA") ? 1 : 0};
+  GraphKey key{h, 0, getenv("EXTERND_CONTRACT_NO_TMA") ? 1 : 0};
   cudaGetDevice(&key.dev);
   std::lock_guard<std::mutex> lock(g_graph_mu);
   for (size_t i = 0; i < g_graphs.size(); ++i)

@@ -23,6 +23,9 @@ struct SeqHostArgs {
   uint8_t* trace_flags;
   int64_t* stats;
   int64_t wait_budget;
+  unsigned flags;         // EXTERND_TSTAT_MEAN_ABS | EXTERND_VSTEP_NAIVE
+  int sweeps;             // refinement sweeps after the greedy pass
+  double* sweep_energy;   // [sweeps] out (device), may be NULL when sweeps == 0
 };
 
 struct BlockHostArgs {
@@ -41,6 +44,7 @@ struct BlockHostArgs {
   const int64_t* trace_block;  // host array: traced block indices
   uint64_t* trace_uv;          // device: per traced block, V0 then U_t, V_t masks
   int32_t* trace_rows;         // device: per traced block, the start rows
+  unsigned flags;              // EXTERND_TSTAT_MEAN_ABS | EXTERND_VSTEP_NAIVE
 };
 
 int seq_decompose(const SeqHostArgs& h, cudaStream_t st);

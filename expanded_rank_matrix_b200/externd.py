@@ -26,10 +26,15 @@ ERR_TIMEOUT = -5
 ERR_NONFINITE = -6
 ERR_SCRATCH_LIMIT = -7
 
+# variant flags of externd_decompose_ex
+TSTAT_MEAN_ABS = 1
+VSTEP_NAIVE = 2
+MAX_SWEEPS = 64
+
 # every symbol include/externd.h declares
-EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_traced",
+EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_ex", "externd_decompose_traced",
            "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc",
-           "externd_decompose_block_traced")
+           "externd_decompose_block_traced", "externd_rank_for_energy")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -55,8 +60,13 @@ def load(path: str = LIB_PATH):
     L.externd_decompose.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float, ctypes.c_int,
                                     _vp, ctypes.c_int, _vp, _vp, _vp, _vp, _vp]
     L.externd_decompose.restype = ctypes.c_int
+    L.externd_decompose_ex.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
+                                       ctypes.c_int, _vp, ctypes.c_int, ctypes.c_uint, ctypes.c_int,
+                                       _vp, _vp, _vp, _vp, _vp, _vp]
+    L.externd_decompose_ex.restype = ctypes.c_int
     L.externd_decompose_traced.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
-                                           ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp, _vp,
+                                           ctypes.c_int, _vp, ctypes.c_int, ctypes.c_uint,
+                                           ctypes.c_int, _vp, _vp, _vp, _vp, _vp,
                                            _i64, _vp, _vp, _vp, _vp, _vp, _i64, _vp]
     L.externd_decompose_traced.restype = ctypes.c_int
     L.externd_reconstruct.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]
@@ -65,9 +75,11 @@ def load(path: str = LIB_PATH):
                                             ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp]
     L.externd_decompose_noalloc.restype = ctypes.c_int
     L.externd_decompose_block_traced.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
-                                                 ctypes.c_int, _vp, ctypes.c_int, _vp, _vp, _vp,
-                                                 _vp, _i64, _vp, _vp, _vp, _vp]
+                                                 ctypes.c_int, _vp, ctypes.c_int, ctypes.c_uint,
+                                                 _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
     L.externd_decompose_block_traced.restype = ctypes.c_int
+    L.externd_rank_for_energy.argtypes = [_vp, _i64, ctypes.c_double, _vp, _vp]
+    L.externd_rank_for_energy.restype = ctypes.c_int
     L.externd_sync_status.argtypes = [_vp]
     L.externd_sync_status.restype = ctypes.c_int
     _lib = L
@@ -103,9 +115,10 @@ class Factors:
     packed_B: torch.Tensor  # int32 view of uint32 [k, 2, ceil(m/32)]
     packed_C: torch.Tensor  # [k, 2, ceil(n/32)]
     D: torch.Tensor         # fp32 [k]
-    energy: torch.Tensor    # fp64 [k]
+    energy: torch.Tensor    # fp64 [k] (the greedy pass)
     m: int
     n: int
+    sweep_energy: Optional[torch.Tensor] = None  # fp64 [sweeps]: after each refinement sweep
 
     @property
     def k(self) -> int:
@@ -121,19 +134,31 @@ def alloc_factors(m: int, n: int, k: int, device) -> Factors:
 
 def decompose_into(out: Factors, A: torch.Tensor, mu: float, tau: float, iters: int,
                    w: Optional[torch.Tensor] = None, block: int = 1,
-                   stream: Optional[torch.cuda.Stream] = None) -> None:
-    """Runs externd_decompose into preallocated outputs (stream ordered)."""
+                   stream: Optional[torch.cuda.Stream] = None, flags: int = 0,
+                   sweeps: int = 0) -> None:
+    """Runs externd_decompose (externd_decompose_ex with variant flags or
+    refinement sweeps) into preallocated outputs (stream ordered)."""
     m, n = A.shape
-    rc = load().externd_decompose(_ptr(A), m, n, mu, tau, iters, _ptr(w), block,
-                                  _ptr(out.packed_B), _ptr(out.packed_C), _ptr(out.D),
-                                  _ptr(out.energy), _stream(stream))
+    if flags == 0 and sweeps == 0:
+        rc = load().externd_decompose(_ptr(A), m, n, mu, tau, iters, _ptr(w), block,
+                                      _ptr(out.packed_B), _ptr(out.packed_C), _ptr(out.D),
+                                      _ptr(out.energy), _stream(stream))
+    else:
+        if sweeps > 0 and (out.sweep_energy is None or out.sweep_energy.numel() < sweeps):
+            out.sweep_energy = torch.empty(sweeps, dtype=torch.float64, device=out.D.device)
+        rc = load().externd_decompose_ex(_ptr(A), m, n, mu, tau, iters, _ptr(w), block, flags,
+                                         sweeps, _ptr(out.packed_B), _ptr(out.packed_C),
+                                         _ptr(out.D), _ptr(out.energy),
+                                         _ptr(out.sweep_energy) if sweeps > 0 else None,
+                                         _stream(stream))
     if rc != OK:
         raise ExterndError(rc, "externd_decompose")
 
 
 def decompose(A: torch.Tensor, mu: float, tau: float, iters: int,
               w: Optional[torch.Tensor] = None, block: int = 1,
-              stream: Optional[torch.cuda.Stream] = None, check: bool = True) -> Factors:
+              stream: Optional[torch.cuda.Stream] = None, check: bool = True, flags: int = 0,
+              sweeps: int = 0) -> Factors:
     if A.dtype != torch.float32 or A.dim() != 2:
         raise ValueError("A must be a 2-D fp32 CUDA tensor")
     m, n = A.shape
@@ -141,7 +166,7 @@ def decompose(A: torch.Tensor, mu: float, tau: float, iters: int,
     if k < 1:
         raise ExterndError(ERR_INVALID_ARG, "externd_rank")
     out = alloc_factors(m, n, k, A.device)
-    decompose_into(out, A, mu, tau, iters, w, block, stream)
+    decompose_into(out, A, mu, tau, iters, w, block, stream, flags, sweeps)
     if check:
         st = sync_status(stream)
         if st != OK:
@@ -173,11 +198,17 @@ class Trace:
 def decompose_traced(A: torch.Tensor, mu: float, tau: float, iters: int,
                      trace_comps: Sequence[int], w: Optional[torch.Tensor] = None,
                      wait_budget: int = 0, stream: Optional[torch.cuda.Stream] = None,
-                     check: bool = True):
+                     check: bool = True, flags: int = 0, sweeps: int = 0):
+    """Traced sequential run.  trace_comps are step indices: component c of
+    the greedy pass is step c, component l's refit in sweep s is step
+    k (1 + s) + l."""
     m, n = A.shape
     k = rank(m, n, mu)
     out = alloc_factors(m, n, k, A.device)
-    comps = np.array(sorted(set(int(c) for c in trace_comps if 0 <= c < k)), dtype=np.int64)
+    if sweeps > 0:
+        out.sweep_energy = torch.empty(sweeps, dtype=torch.float64, device=A.device)
+    nsteps = k * (1 + sweeps)
+    comps = np.array(sorted(set(int(c) for c in trace_comps if 0 <= c < nsteps)), dtype=np.int64)
     nt = int(comps.size)
     S = 2 * words(n) + iters * 2 * (words(m) + words(n))
     dev = A.device
@@ -187,8 +218,9 @@ def decompose_traced(A: torch.Tensor, mu: float, tau: float, iters: int,
     tf = torch.zeros(max(nt, 1), dtype=torch.uint8, device=dev)
     stats = torch.zeros(16, dtype=torch.int64, device=dev)
     rc = load().externd_decompose_traced(
-        _ptr(A), m, n, mu, tau, iters, _ptr(w), 1, _ptr(out.packed_B), _ptr(out.packed_C),
-        _ptr(out.D), _ptr(out.energy), nt, _ptr(tc), _ptr(tb) if nt else None,
+        _ptr(A), m, n, mu, tau, iters, _ptr(w), 1, flags, sweeps, _ptr(out.packed_B),
+        _ptr(out.packed_C), _ptr(out.D), _ptr(out.energy),
+        _ptr(out.sweep_energy) if sweeps > 0 else None, nt, _ptr(tc), _ptr(tb) if nt else None,
         _ptr(tr) if nt else None, _ptr(tf) if nt else None, _ptr(stats), wait_budget,
         _stream(stream))
     if rc != OK:
@@ -206,6 +238,39 @@ def reconstruct(f: Factors, stream: Optional[torch.cuda.Stream] = None) -> torch
     if rc != OK:
         raise ExterndError(rc, "externd_reconstruct")
     return out
+
+
+def rank_for_energy(energy: torch.Tensor, target: float,
+                    stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Smallest rank whose prefix of a sequential decomposition reaches the
+    energy target (0: none does), found by externd_rank_for_energy."""
+    if energy.dtype != torch.float64 or energy.dim() != 1:
+        raise ValueError("energy must be a 1-D fp64 CUDA tensor")
+    out = torch.empty(1, dtype=torch.int64, device=energy.device)
+    rc = load().externd_rank_for_energy(_ptr(energy), energy.shape[0], float(target), _ptr(out),
+                                        _stream(stream))
+    if rc != OK:
+        raise ExterndError(rc, "externd_rank_for_energy")
+    return int(out.item())
+
+
+def truncate(f: Factors, r: int) -> Factors:
+    """The first r components (views): the rank-r decomposition of a
+    sequential run, since greedy deflation is prefix-consistent."""
+    return Factors(f.packed_B[:r], f.packed_C[:r], f.D[:r], f.energy[:r], f.m, f.n)
+
+
+def allocate_rank(A: torch.Tensor, target: float, mu_max: float, tau: float, iters: int,
+                  w: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None):
+    """Per-matrix rank allocation: decomposes A sequentially at mu_max and
+    returns (rank, mu, factors) for the smallest rank reaching `target`
+    (rank 0 and the full factors when even mu_max falls short)."""
+    f = decompose(A, mu_max, tau, iters, w=w, block=1, stream=stream)
+    r = rank_for_energy(f.energy, target, stream)
+    if r == 0:
+        return 0, mu_max, f
+    return r, r / min(f.m, f.n), truncate(f, r)
 
 
 def sync_status(stream: Optional[torch.cuda.Stream] = None) -> int:
@@ -256,7 +321,8 @@ class BlockTrace:
 
 def decompose_block_traced(A: torch.Tensor, mu: float, tau: float, iters: int, block: int,
                            trace_blocks: Sequence[int], w: Optional[torch.Tensor] = None,
-                           stream: Optional[torch.cuda.Stream] = None, check: bool = True):
+                           stream: Optional[torch.cuda.Stream] = None, check: bool = True,
+                           flags: int = 0):
     m, n = A.shape
     k = rank(m, n, mu)
     out = alloc_factors(m, n, k, A.device)
@@ -267,7 +333,8 @@ def decompose_block_traced(A: torch.Tensor, mu: float, tau: float, iters: int, b
     uv = torch.zeros((max(nt, 1), words_), dtype=torch.int64, device=A.device)
     rows = torch.zeros((max(nt, 1), block), dtype=torch.int32, device=A.device)
     rc = load().externd_decompose_block_traced(
-        _ptr(A), m, n, mu, tau, iters, _ptr(w), block, _ptr(out.packed_B), _ptr(out.packed_C),
+        _ptr(A), m, n, mu, tau, iters, _ptr(w), block, flags, _ptr(out.packed_B),
+        _ptr(out.packed_C),
         _ptr(out.D), _ptr(out.energy), nt,
         blocks.ctypes.data_as(ctypes.c_void_p) if nt else None, _ptr(uv) if nt else None,
         _ptr(rows) if nt else None, _stream(stream))

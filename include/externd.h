@@ -48,6 +48,21 @@ extern "C" {
 typedef struct CUstream_st* externd_stream_t; /* same object as cudaStream_t */
 
 /*
+ * Variant flags of externd_decompose_ex (the threshold and V-step options the
+ * romaanj.github.io review names in "Method" and "Validation").
+ *
+ * EXTERND_TSTAT_MEAN_ABS: T_tau(x)_j = sign(x_j) if |x_j| > tau * mean_j |x_j|
+ *   (instead of tau * rms(x)).  The review's zero shares (tau = 0.7 -> ~41%,
+ *   tau = 2.0 -> ~87%) are those of this statistic on Gaussian data.
+ * EXTERND_VSTEP_NAIVE: with weights, the V-step thresholds W R^T u (the
+ *   "naive" importance-weighted V-step of the review's ablation) instead of
+ *   R^T u (the corrected one, the default).  No effect without weights.
+ */
+#define EXTERND_TSTAT_MEAN_ABS 1u
+#define EXTERND_VSTEP_NAIVE 2u
+#define EXTERND_MAX_SWEEPS 64
+
+/*
  * externd_rank -- the inner rank k = floor(mu * min(m, n)) (the paper's
  * abstract: k = mu min(m, n)).  Returns 0 when an argument is out of range.
  */
@@ -106,19 +121,49 @@ int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau,
                       float* D, double* energy_trace, externd_stream_t stream);
 
 /*
- * externd_decompose_traced -- externd_decompose plus a record of the ALS
- * trajectory of selected components (used to compare the device path with a
- * reference half-step by half-step).  Sequential mode (block == 1) only.
+ * externd_decompose_ex -- externd_decompose with the threshold variants and
+ * refinement sweeps.
  *
- *   trace_comp   [ntrace] int64, strictly increasing component indices, or
- *                NULL when ntrace == 0.
+ *   flags        EXTERND_TSTAT_MEAN_ABS | EXTERND_VSTEP_NAIVE, or 0 (the
+ *                externd_decompose behaviour).  Both modes.
+ *   sweeps       refinement sweeps after the greedy pass, 0 .. EXTERND_MAX_SWEEPS;
+ *                block == 1 only.  A sweep backfits every component in order
+ *                (the review's "Results": sweeps add about 0.4 energy points):
+ *                component l is added back onto the residual, refit by
+ *                `iters` ALS rounds from its own v, and replaced by the refit
+ *                only if the refit removes more than the old pattern with its
+ *                scale re-solved on that residual (otherwise the old pattern
+ *                stays, rescaled); the single-entry safeguard applies as in
+ *                the greedy pass.  No step raises the residual beyond fp32
+ *                rounding.  The outputs then hold the refined factors;
+ *                energy_trace keeps the greedy pass's trace.
+ *   sweep_energy [sweeps] fp64 out: the energy after each sweep (NULL when
+ *                sweeps == 0).
+ * Other arguments, scratch and errors as for externd_decompose (sweeps add
+ * 4 * k bytes per CTA of the persistent grid to the stream-ordered scratch).
+ */
+int externd_decompose_ex(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
+                         const float* w, int block, unsigned flags, int sweeps,
+                         uint32_t* packed_B, uint32_t* packed_C, float* D, double* energy_trace,
+                         double* sweep_energy, externd_stream_t stream);
+
+/*
+ * externd_decompose_traced -- externd_decompose_ex plus a record of the ALS
+ * trajectory of selected steps (used to compare the device path with a
+ * reference half-step by half-step).  Tracing is sequential-mode
+ * (block == 1) only.  Step t < k is greedy component t; step k (1 + s) + l
+ * is component l's refit in sweep s.
+ *
+ *   trace_comp   [ntrace] int64, strictly increasing step indices below
+ *                k (1 + sweeps), or NULL when ntrace == 0.
  *   trace_bits   [ntrace][S] uint32 out, S = 2*Wn + iters*2*(Wm + Wn),
  *                Wm = ceil(m/32), Wn = ceil(n/32): for each traced component
- *                the packed starting v, then for t = 1..iters the packed u_t
- *                and the packed v_t.  May be NULL when ntrace == 0.
- *   trace_row    [ntrace] int32 out: the starting row i*.
+ *                the packed starting v (a refit's: the old component's v),
+ *                then for t = 1..iters the packed u_t and the packed v_t.
+ *                May be NULL when ntrace == 0.
+ *   trace_row    [ntrace] int32 out: the starting row i* (-1 for a refit).
  *   trace_flags  [ntrace] uint8 out: bit 0 = the safeguard replaced the ALS
- *                pair of this component.
+ *                pair of this step, bit 1 = a refit kept the old pattern.
  *   stats        [16] int64 out or NULL: [0] safeguard activations over all
  *                components, [1] components emitted as zero because the
  *                residual vanished, [2] launch clusters, [3] CTAs per cluster,
@@ -133,14 +178,16 @@ int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau,
  *                winds down without further waits.
  */
 int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
-                             const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
-                             float* D, double* energy_trace, int64_t ntrace,
+                             const float* w, int block, unsigned flags, int sweeps,
+                             uint32_t* packed_B, uint32_t* packed_C, float* D,
+                             double* energy_trace, double* sweep_energy, int64_t ntrace,
                              const int64_t* trace_comp, uint32_t* trace_bits, int32_t* trace_row,
                              uint8_t* trace_flags, int64_t* stats, int64_t wait_budget,
                              externd_stream_t stream);
 
 /*
- * externd_decompose_block_traced -- externd_decompose with block >= 2 plus a
+ * externd_decompose_block_traced -- externd_decompose_ex with block >= 2
+ * (flags as there, no sweeps) plus a
  * record of the block-ALS trajectory of selected blocks (used to compare the
  * device path with a reference half-step by half-step).  Block t covers
  * components t*block .. min(k, (t+1)*block) - 1; bit l of a mask word stands
@@ -156,7 +203,8 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
  *                order (energy descending, index ascending).
  */
 int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float mu, float tau,
-                                   int iters, const float* w, int block, uint32_t* packed_B,
+                                   int iters, const float* w, int block, unsigned flags,
+                                   uint32_t* packed_B,
                                    uint32_t* packed_C, float* D, double* energy_trace,
                                    int64_t ntrace, const int64_t* trace_block, uint64_t* trace_uv,
                                    int32_t* trace_rows, externd_stream_t stream);
@@ -205,6 +253,30 @@ int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, cons
 int externd_decompose_noalloc(const float* A, int64_t m, int64_t n, float mu, float tau,
                               int iters, const float* w, uint32_t* packed_B, uint32_t* packed_C,
                               float* D, double* energy_trace, externd_stream_t stream);
+
+/*
+ * externd_rank_for_energy -- per-matrix rank allocation to an energy target
+ * (the romaanj.github.io review, "Results": the rank multiplier is chosen per
+ * matrix to reach a reference quantiser's per-matrix energy; the Pith
+ * review's "Assumptions & free parameters": mu from 1.97 to 3.43 per matrix).
+ * Greedy sequential deflation (block == 1) makes a rank-k decomposition hold
+ * every shorter one as its prefix, bit for bit, so the smallest rank whose
+ * energy reaches `target` is read off one run's energy trace: the first c
+ * with energy_trace[c] >= target, plus one.  The first r components of
+ * packed_B, packed_C and D are then exactly the rank-r decomposition.  (In
+ * block mode a prefix is a shorter run only where it ends on a block
+ * boundary.)
+ *
+ *   energy_trace [k] fp64 (device) in, as written by externd_decompose.
+ *   k            >= 1 entries.
+ *   target       finite energy target (e.g. 0.994).
+ *   rank         [1] int64 (device) out: that rank in 1..k, or 0 when no
+ *                prefix reaches the target.
+ * Stream-ordered on `stream`; returns EXTERND_OK, EXTERND_ERR_INVALID_ARG
+ * (NULL or misaligned pointer, k < 1, target not finite) or EXTERND_ERR_CUDA.
+ */
+int externd_rank_for_energy(const double* energy_trace, int64_t k, double target, int64_t* rank,
+                            externd_stream_t stream);
 
 /*
  * externd_sync_status -- synchronises `stream`, then returns and clears the

@@ -68,10 +68,31 @@ def test_host_argument_checks(lib):
     assert L.externd_reconstruct(nul, fake, fake, 4, 4, 4, fake, nul) == X.ERR_INVALID_ARG
     assert L.externd_reconstruct(fake, fake, fake, 4, 4, 0, fake, nul) == X.ERR_INVALID_ARG
     # tracing is a sequential-mode feature and needs its buffers
-    assert L.externd_decompose_traced(fake, 8, 8, 1.0, 0.5, 2, nul, 1, fake, fake, fake, fake, 2,
-                                      nul, nul, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
-    assert L.externd_decompose_traced(fake, 8, 8, 1.0, 0.5, 2, nul, 1, fake, fake, fake, fake, 0,
-                                      nul, nul, nul, nul, nul, -1, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_traced(fake, 8, 8, 1.0, 0.5, 2, nul, 1, 0, 0, fake, fake, fake, fake,
+                                      nul, 2, nul, nul, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_traced(fake, 8, 8, 1.0, 0.5, 2, nul, 1, 0, 0, fake, fake, fake, fake,
+                                      nul, 0, nul, nul, nul, nul, nul, -1, nul) == X.ERR_INVALID_ARG
+
+
+def test_variant_and_sweep_argument_checks(lib):
+    L = lib
+    nul = None
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: rejected before any CUDA call
+    ok_flags = X.TSTAT_MEAN_ABS | X.VSTEP_NAIVE
+    # unknown flag bits
+    assert L.externd_decompose_ex(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 4, 0, fake, fake, fake, fake,
+                                  nul, nul) == X.ERR_INVALID_ARG
+    # sweeps: sequential mode only, bounded, and they need their energy output
+    assert L.externd_decompose_ex(fake, 64, 64, 1.0, 0.5, 2, nul, 16, ok_flags, 1, fake, fake,
+                                  fake, fake, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_ex(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 0, -1, fake, fake, fake,
+                                  fake, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_ex(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 0, X.MAX_SWEEPS + 1, fake,
+                                  fake, fake, fake, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_ex(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 0, 2, fake, fake, fake, fake,
+                                  nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, 8, fake, fake,
+                                            fake, fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
 
 
 def test_block_argument_checks(lib):
@@ -84,14 +105,14 @@ def test_block_argument_checks(lib):
     assert L.externd_decompose(fake, 40, 30, 1.0, 0.5, 2, nul, 31, fake, fake, fake, fake,
                                nul) == X.ERR_INVALID_ARG
     # the block-traced entry is block-mode only and needs its trace buffers
-    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 1, fake, fake, fake,
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 0, fake, fake, fake,
                                             fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
-    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, fake, fake, fake,
-                                            fake, 2, nul, nul, nul, nul) == X.ERR_INVALID_ARG
-    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, fake, fake, fake,
-                                            fake, -1, nul, nul, nul, nul) == X.ERR_INVALID_ARG
-    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 65, fake, fake, fake,
-                                            fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, 0, fake, fake,
+                                            fake, fake, 2, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, 0, fake, fake,
+                                            fake, fake, -1, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 65, 0, fake, fake,
+                                            fake, fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
 
 
 def test_unpack_planes_layout():
@@ -106,3 +127,15 @@ def test_unpack_planes_layout():
     expect = np.zeros(40, np.int8)
     expect[0], expect[1], expect[33] = 1, -1, 1
     assert np.array_equal(codes, expect)
+
+
+def test_rank_for_energy_argument_checks(lib):
+    L = lib
+    nul = None
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.externd_rank_for_energy(nul, 4, 0.5, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_rank_for_energy(fake, 4, 0.5, nul, nul) == X.ERR_INVALID_ARG
+    assert L.externd_rank_for_energy(fake, 0, 0.5, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_rank_for_energy(fake, 4, float("nan"), fake, nul) == X.ERR_INVALID_ARG
+    mis = ctypes.c_void_p((1 << 20) + 4)  # fp64 / int64 need 8-byte alignment
+    assert L.externd_rank_for_energy(mis, 4, 0.5, fake, nul) == X.ERR_INVALID_ARG
