@@ -660,4 +660,31 @@ void orc_decompose_block(const float* A, int64_t m, int64_t n, int64_t k, double
   orc_decompose_block2(A, m, n, k, tau, iters, w, 0, b, U, V, D, energy, init_row);
 }
 
+// Inference with the factors ([REV] "Significance": inference stays
+// multiplication-free -- ternary adds and subtracts plus one scale per
+// component; "Limitations" / "Future work": a fused inference kernel is the
+// missing piece): for each of the nb input vectors x (rows of X, nb x n),
+// t_c = sum_j C_cj x_j, then y_i = sum_c B_ic D_c t_c, in fp64.  U is k x m
+// (row c = column c of B), V is k x n (row c of C); Y is nb x m.
+void orc_ternary_apply(const int8_t* U, const int8_t* V, const float* D, int64_t m, int64_t n,
+                       int64_t k, const float* X, int64_t nb, double* Y) {
+  std::vector<double> t(k);
+  for (int64_t b = 0; b < nb; ++b) {
+    const float* x = X + b * n;
+    for (int64_t c = 0; c < k; ++c) {
+      double s = 0.0;
+      for (int64_t j = 0; j < n; ++j)
+        if (V[c * n + j]) s += (double)V[c * n + j] * (double)x[j];
+      t[c] = s;
+    }
+    double* y = Y + b * m;
+    for (int64_t i = 0; i < m; ++i) y[i] = 0.0;
+    for (int64_t c = 0; c < k; ++c) {
+      const double sc = (double)D[c] * t[c];
+      for (int64_t i = 0; i < m; ++i)
+        if (U[c * m + i]) y[i] += (double)U[c * m + i] * sc;
+    }
+  }
+}
+
 }  // extern "C"

@@ -81,6 +81,8 @@ def lib():
         L.orc_reconstruct.restype = None
         L.orc_rank_for_energy.argtypes = [_D, _i64, ctypes.c_double]
         L.orc_rank_for_energy.restype = _i64
+        L.orc_ternary_apply.argtypes = [_I8, _I8, _F, _i64, _i64, _i64, _F, _i64, _D]
+        L.orc_ternary_apply.restype = None
         L.orc_top_rows.argtypes = [_D, _i64, _i64, _I64]
         L.orc_top_rows.restype = None
         L.orc_block_u_step.argtypes = [_F, _i64, _i64, _i64, _I8, _F, ctypes.c_double, _I8, _D, _D]
@@ -295,6 +297,19 @@ def rank_for_energy(energy, target: float) -> int:
     """Smallest rank r whose prefix reaches the energy target (0: none)."""
     e = np.ascontiguousarray(energy, np.float64)
     return int(lib().orc_rank_for_energy(_p(e, _D), e.shape[0], target))
+
+
+def ternary_apply(U, V, D, X) -> np.ndarray:
+    """Y = X (B diag(D) C)^T for the nb x n inputs X (fp64 result, nb x m)."""
+    U = np.ascontiguousarray(U, np.int8); V = np.ascontiguousarray(V, np.int8)
+    D = _f32(D)
+    X = np.ascontiguousarray(np.atleast_2d(X), np.float32)
+    k, m = U.shape
+    n = V.shape[1]
+    nb = X.shape[0]
+    Y = np.empty((nb, m))
+    lib().orc_ternary_apply(_p(U, _I8), _p(V, _I8), _p(D, _F), m, n, k, _p(X, _F), nb, _p(Y, _D))
+    return Y
 
 
 def top_rows(rho, b: int):

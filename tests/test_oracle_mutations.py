@@ -50,6 +50,9 @@ MUTATIONS = [
      "d = D[l];"),
     ("sweep_single_entry_ignores_old", "const double g_best = sc[5] > g_old ? sc[5] : g_old;",
      "const double g_best = sc[5];"),
+    ("apply_drops_scale", "const double sc = (double)D[c] * t[c];", "const double sc = t[c];"),
+    ("apply_sign_dropped", "if (V[c * n + j]) s += (double)V[c * n + j] * (double)x[j];",
+     "if (V[c * n + j]) s += (double)x[j];"),
 ]
 
 PIN_TESTS = [
@@ -78,6 +81,8 @@ PIN_TESTS = [
     lambda o: pins.test_sweep_steps_match_a_replay_by_hand(o, False),
     lambda o: pins.test_sweep_steps_match_a_replay_by_hand(o, True),
     pins.test_sweeps_never_raise_the_residual,
+    pins.test_ternary_apply_against_numpy_and_the_reconstruction,
+    pins.test_ternary_apply_exact_on_integers,
 ]
 
 

@@ -632,3 +632,33 @@ def test_sweeps_keep_exact_components(oracle):
     dec = oracle.decompose(A, 3, 0.5, 3, sweeps=2)
     assert np.all(dec.sweep_energy == 1.0)
     assert abs(dec.D[0]) == 2.0 and abs(dec.D[1]) == 0.5
+
+
+# --- inference with the factors ------------------------------------------------
+
+def test_ternary_apply_against_numpy_and_the_reconstruction(oracle):
+    """y = B diag(D) C x: against numpy's matmul of the unpacked factors, and
+    against the dense reconstruction times x."""
+    A = W.llm_like(48, 40, 67, n_outliers=2)
+    dec = oracle.decompose(A, 80, 0.5, 3)
+    rng = _rng(71)
+    X = rng.standard_normal((3, 40)).astype(np.float32)
+    Y = oracle.ternary_apply(dec.U, dec.V, dec.D, X)
+    B = dec.U.T.astype(np.float64)
+    C = dec.V.astype(np.float64)
+    ref = (B @ (dec.D.astype(np.float64)[:, None] * (C @ X.T.astype(np.float64)))).T
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+    Ahat = oracle.reconstruct(dec.U, dec.V, dec.D, 48, 40)
+    assert np.allclose(Y, X.astype(np.float64) @ Ahat.T, rtol=1e-10, atol=1e-10)
+
+
+def test_ternary_apply_exact_on_integers(oracle):
+    """Two ternary components with integer scales and an integer input: the
+    result is a small integer vector known by hand."""
+    U = np.array([[1, 0, -1], [0, 1, 1]], np.int8)          # B^T: 2 components, m = 3
+    V = np.array([[1, -1, 0, 1], [0, 1, 1, 0]], np.int8)    # C: n = 4
+    D = np.array([2.0, -3.0], np.float32)
+    x = np.array([[1.0, 2.0, 3.0, 4.0]], np.float32)
+    # t = (1 - 2 + 4, 2 + 3) = (3, 5); s = (6, -15); y = (6, -15, -6 - 15)
+    Y = oracle.ternary_apply(U, V, D, x)
+    assert Y.tolist() == [[6.0, -15.0, -21.0]]
