@@ -126,6 +126,19 @@ int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, cons
   return externd::reconstruct(packed_B, packed_C, D, m, n, k, A_hat, (cudaStream_t)stream);
 }
 
+int externd_ternary_apply(const uint32_t* packed_B, const uint32_t* packed_C, const float* D,
+                          int64_t m, int64_t n, int64_t k, const float* X, int64_t nb, float* Y,
+                          externd_stream_t stream) {
+  if (!packed_B || !packed_C || !D || !X || !Y) return EXTERND_ERR_INVALID_ARG;
+  if (!aligned4(packed_B) || !aligned4(packed_C) || !aligned4(D) || !aligned4(X) || !aligned4(Y))
+    return EXTERND_ERR_INVALID_ARG;
+  if (!sizes_ok(m, n) || m > EXTERND_APPLY_MAX_ROWS || k < 1 || k > 2147483647LL)
+    return EXTERND_ERR_INVALID_ARG;
+  if (nb < 1 || nb > 65536 || nb * (m > n ? m : n) >= ((int64_t)1 << 31))
+    return EXTERND_ERR_INVALID_ARG;
+  return externd::ternary_apply(packed_B, packed_C, D, m, n, k, X, nb, Y, (cudaStream_t)stream);
+}
+
 int externd_sync_status(externd_stream_t stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return EXTERND_ERR_CUDA;
   int* p = externd::status_word_ptr();

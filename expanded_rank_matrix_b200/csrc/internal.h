@@ -52,6 +52,8 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st);
 int reconstruct(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
                 int64_t k, float* out, cudaStream_t st);
 int* status_word_ptr();
+int ternary_apply(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
+                  int64_t k, const float* X, int64_t nb, float* Y, cudaStream_t st);
 // Block-ALS contractions on the tensor cores.  Vm/Vs (Um/Us) are the 64-bit
 // per-entry masks of the ternary operand, Bop the same codes as bf16 B chunks
 // (4 KB per 32 entries); wpad the weights zero padded to a multiple of 32.

@@ -34,7 +34,8 @@ MAX_SWEEPS = 64
 # every symbol include/externd.h declares
 EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_ex", "externd_decompose_traced",
            "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc",
-           "externd_decompose_block_traced", "externd_rank_for_energy")
+           "externd_decompose_block_traced", "externd_rank_for_energy",
+           "externd_ternary_apply")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -80,6 +81,8 @@ def load(path: str = LIB_PATH):
     L.externd_decompose_block_traced.restype = ctypes.c_int
     L.externd_rank_for_energy.argtypes = [_vp, _i64, ctypes.c_double, _vp, _vp]
     L.externd_rank_for_energy.restype = ctypes.c_int
+    L.externd_ternary_apply.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp]
+    L.externd_ternary_apply.restype = ctypes.c_int
     L.externd_sync_status.argtypes = [_vp]
     L.externd_sync_status.restype = ctypes.c_int
     _lib = L
@@ -271,6 +274,24 @@ def allocate_rank(A: torch.Tensor, target: float, mu_max: float, tau: float, ite
     if r == 0:
         return 0, mu_max, f
     return r, r / min(f.m, f.n), truncate(f, r)
+
+
+def apply_into(f: Factors, X: torch.Tensor, Y: torch.Tensor,
+               stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Y = X (B diag(D) C)^T from the packed factors (externd_ternary_apply);
+    X is [nb, n] fp32, Y [nb, m] fp32, both on the device."""
+    nb = X.shape[0]
+    rc = load().externd_ternary_apply(_ptr(f.packed_B), _ptr(f.packed_C), _ptr(f.D), f.m, f.n, f.k,
+                                      _ptr(X), nb, _ptr(Y), _stream(stream))
+    if rc != OK:
+        raise ExterndError(rc, "externd_ternary_apply")
+
+
+def apply(f: Factors, X: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    X2 = X.reshape(-1, f.n).contiguous()
+    Y = torch.empty((X2.shape[0], f.m), dtype=torch.float32, device=X.device)
+    apply_into(f, X2, Y, stream)
+    return Y.reshape(*X.shape[:-1], f.m)
 
 
 def sync_status(stream: Optional[torch.cuda.Stream] = None) -> int:

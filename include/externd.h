@@ -220,6 +220,34 @@ int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, cons
                         int64_t m, int64_t n, int64_t k, float* A_hat, externd_stream_t stream);
 
 /*
+ * externd_ternary_apply -- inference with the factors: Y = X (B diag(D) C)^T
+ * from the packed bitplanes, without forming the dense matrix.  For each
+ * input vector x (a row of X): t_c = sum_j C_cj x_j, then
+ * y_i = sum_c B_ic D_c t_c -- ternary additions and subtractions plus one
+ * scale per component (the romaanj.github.io review, "Significance":
+ * inference stays multiplication-free; "Limitations": no fused inference
+ * kernel exists yet).  Sums are fp32 in a fixed order (reproducible run to
+ * run).
+ *
+ *   packed_B [k][2][ceil(m/32)], packed_C [k][2][ceil(n/32)], D [k]: the
+ *            factors as externd_decompose writes them (device, in).
+ *   m, n, k  1 <= m <= EXTERND_APPLY_MAX_ROWS, 1 <= n, m*n < 2^31, k >= 1.
+ *   X        [nb][n] fp32 (device, in): nb input vectors, row-major.
+ *   nb       1 .. 65536 vectors (processed two at a time).
+ *   Y        [nb][m] fp32 (device, out).
+ * Scratch (k + SMs * m) * 2 floats, stream-ordered on `stream` like
+ * externd_decompose's.  One cooperative launch per two vectors (every CTA
+ * resident; its two grid barriers are bounded waits that raise
+ * EXTERND_ERR_TIMEOUT in the status word if they ever run out).  Returns
+ * EXTERND_OK, EXTERND_ERR_INVALID_ARG, EXTERND_ERR_OOM, EXTERND_ERR_NO_COOP
+ * or EXTERND_ERR_CUDA.
+ */
+#define EXTERND_APPLY_MAX_ROWS 16384
+int externd_ternary_apply(const uint32_t* packed_B, const uint32_t* packed_C, const float* D,
+                          int64_t m, int64_t n, int64_t k, const float* X, int64_t nb, float* Y,
+                          externd_stream_t stream);
+
+/*
  * externd_decompose_noalloc -- externd_decompose (block == 1 only) without
  * any memory allocation.  The paper has no counterpart; this is a service of
  * this library.

@@ -139,3 +139,16 @@ def test_rank_for_energy_argument_checks(lib):
     assert L.externd_rank_for_energy(fake, 4, float("nan"), fake, nul) == X.ERR_INVALID_ARG
     mis = ctypes.c_void_p((1 << 20) + 4)  # fp64 / int64 need 8-byte alignment
     assert L.externd_rank_for_energy(mis, 4, 0.5, fake, nul) == X.ERR_INVALID_ARG
+
+
+def test_ternary_apply_argument_checks(lib):
+    L = lib
+    nul = None
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.externd_ternary_apply(nul, fake, fake, 8, 8, 4, fake, 1, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_ternary_apply(fake, fake, fake, 8, 8, 0, fake, 1, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_ternary_apply(fake, fake, fake, 8, 8, 4, fake, 0, fake, nul) == X.ERR_INVALID_ARG
+    assert L.externd_ternary_apply(fake, fake, fake, 16385, 8, 4, fake, 1, fake,
+                                   nul) == X.ERR_INVALID_ARG  # more rows than one launch covers
+    mis = ctypes.c_void_p((1 << 20) + 2)
+    assert L.externd_ternary_apply(fake, fake, fake, 8, 8, 4, mis, 1, fake, nul) == X.ERR_INVALID_ARG
