@@ -86,11 +86,17 @@ def test_llm1024_sampled_blocks_and_free_running(oracle):
     assert abs(E[-1] - ref.energy[-1]) <= FREE_ENERGY_ATOL
 
 
-def test_mlp9728_first_blocks(oracle):
+def test_mlp9728_blocks_across_the_run(oracle):
+    """Config 4 (9728 x 2560, mu = 2, I = 4, b = 64): blocks spread over the whole
+    80-block run are teacher-forced -- the oracle replays the device's emitted
+    components up to each one, so late blocks are checked on the residual the
+    ordered deflations and stream-K partials have built up; the energy after
+    block 0 is held to 1e-4 against the stored oracle value."""
     wl = W.config_mlp9728(64)
-    rep, f = block_teacher_forced(oracle, wl.a, wl.mu, wl.tau, wl.iters, 64, blocks=[0, 1])
-    print(f"mlp9728 b=64: band {rep.band_total} mismatch {rep.band_mismatch} "
-          f"max D rel {rep.d_rel_max:.2e}")
+    rep, f = block_teacher_forced(oracle, wl.a, wl.mu, wl.tau, wl.iters, 64,
+                                  blocks=[0, 1, 20, 40, 79])
+    print(f"mlp9728 b=64: blocks {rep.blocks}, band {rep.band_total} mismatch "
+          f"{rep.band_mismatch}, max D rel {rep.d_rel_max:.2e}")
     assert rep.ok, rep.bad
     p = os.path.join(os.path.dirname(__file__), "golden", "oracle_energy.json")
     g = json.load(open(p))["mlp9728_b64"]
@@ -98,6 +104,7 @@ def test_mlp9728_first_blocks(oracle):
     E = f.energy.cpu().numpy()
     print(f"  energy after block 0: device {E[63]:.8f} oracle {g['energy_at']['63']:.8f}; "
           f"final: device {E[-1]:.8f} oracle {g['final_energy']:.8f}")
+    assert abs(E[63] - g["energy_at"]["63"]) <= FREE_ENERGY_ATOL
     assert abs(E[-1] - g["final_energy"]) <= FREE_ENERGY_ATOL_LONG_BLOCK
 
 

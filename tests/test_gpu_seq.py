@@ -220,3 +220,23 @@ def test_attn2560_full_size(oracle):
     f2 = X.decompose(_dev(wl.a), wl.mu, wl.tau, wl.iters)
     assert torch.equal(f2.packed_B, f.packed_B) and torch.equal(f2.packed_C, f.packed_C)
     assert torch.equal(f2.D, f.D) and torch.equal(f2.energy, f.energy)
+
+
+def test_mlp9728_hybrid_residency(oracle):
+    """Config 4 at block = 1 (9728 x 2560, mu = 2, I = 4): the residual does not
+    fit the grid's shared memory, so most rows of every tile stream from
+    global memory (the hybrid kernel).  Sampled components are teacher-forced
+    and the final energy is held to 1e-4 against the oracle's stored run."""
+    wl = W.config_mlp9728(1)
+    g = _golden()["mlp9728_b1"]
+    assert g["k"] == wl.k and g["seed"] == wl.meta["seed"]
+    comps = [0, 1, 100, 2559, 2560, 5119]
+    rep, f, tr = teacher_forced(oracle, wl.a, wl.mu, wl.tau, wl.iters, comps=comps)
+    stats = tr.stats.cpu().numpy()
+    print(f"mlp9728 b=1: plan NC={stats[2]} CS={stats[3]} rows in shared memory {stats[4]} "
+          f"of {stats[5]}; band {rep.band_total} mismatch {rep.band_mismatch} "
+          f"fallbacks {rep.fallbacks}")
+    assert 0 <= stats[4] < stats[5]  # part of every tile lives in global memory
+    assert rep.ok, rep.bad
+    E = f.energy.cpu().numpy()
+    assert abs(E[-1] - g["final_energy"]) <= FREE_ENERGY_ATOL
