@@ -7,7 +7,7 @@ iterations, block = 1) through the C ABI.  Prints one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload attn2560|mlp9728_b64|mlp9728_b1|block_layer]
-  python bench.py --case attn2560_k64|mlp9728_3blocks     (small profiling cases)
+  python bench.py --case attn2560_k64|mlp9728_3blocks|apply_attn2560   (small profiling cases)
 
 --workload picks another configuration (default: the 2560 x 2560 one above);
 mlp9728_b64 / _b1 decompose the 9728 x 2560 MLP-shaped matrix (mu = 2) with
@@ -180,6 +180,80 @@ def _profiled_traffic(kernel: str, workload: str):
         return None
 
 
+def _host_cpu():
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+def _factor_report(f, stats):
+    """Zero shares of B and C, effective bits per weight under the mask+sign
+    storage model (Pith review, "Assumptions & free parameters", Eq. 5: a
+    mask bit per factor entry plus a sign bit per nonzero, i.e. 2 - sparsity
+    bits per entry; the scales D absorbed as the review says), and the
+    safeguard count of the run."""
+    import numpy as np
+    pB = f.packed_B.cpu().numpy().view(np.uint32)
+    pC = f.packed_C.cpu().numpy().view(np.uint32)
+
+    def nnz(planes):
+        return int(np.unpackbits(planes[:, 0, :].view(np.uint8)).sum())
+
+    k, m, n = f.k, f.m, f.n
+    nzB, nzC = nnz(pB), nnz(pC)
+    zB, zC = 1.0 - nzB / (k * m), 1.0 - nzC / (k * n)
+    bits = k * m * (2.0 - zB) + k * n * (2.0 - zC)
+    return {"zero_frac_B": zB, "zero_frac_C": zC, "eff_bpw_eq5": bits / (m * n),
+            "eff_bpw_with_fp32_D": (bits + 32.0 * k) / (m * n),
+            "safeguard_activations": int(stats[0]) if stats is not None else None}
+
+
+def _onchip_peaks(X, dev):
+    """SMEM and L2 read bandwidth (GB/s) measured in this run (best of 3)."""
+    import torch
+    buf = torch.ones(26 << 18, dtype=torch.float32, device=dev)  # 26 MiB, L2-resident
+    X.probe_read_bandwidth(X.PROBE_SMEM, 200)
+    X.probe_read_bandwidth(X.PROBE_L2, 40, buf)
+    # a few milliseconds each, so launch costs do not count
+    smem = max(X.probe_read_bandwidth(X.PROBE_SMEM, 4000) for _ in range(3))
+    l2 = max(X.probe_read_bandwidth(X.PROBE_L2, 400, buf) for _ in range(3))
+    del buf
+    return smem / 1e9, l2 / 1e9
+
+
+def _apply_measure(X, f, dev, flush, peak, reps=20):
+    """The inference kernel on this run's factors: one vector per call, L2
+    flushed before every call, each call timed with events."""
+    import torch
+    x = torch.randn(1, f.n, device=dev)
+    y = torch.empty(1, f.m, device=dev)
+    for _ in range(3):
+        X.apply_into(f, x, y)
+    times = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        X.apply_into(f, x, y)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) / 1000.0)
+    if X.sync_status() != X.OK:
+        raise SystemExit("device status error in the inference measurement")
+    t = statistics.median(times)
+    nbytes = 4.0 * f.k * 2 * ((f.m + 31) // 32 + (f.n + 31) // 32) + 4.0 * (f.k + f.n + f.m)
+    return {"kernel": "apply_kernel (externd_ternary_apply)", "vectors_per_call": 1,
+            "us_per_call": 1e6 * t, "bytes_per_call": nbytes, "achieved_gbs": nbytes / t / 1e9,
+            "frac_of_hbm": nbytes / t / 1e9 / peak, "l2": "flushed before every call",
+            "note": "bytes = packed B and C planes, D, x and y; median of %d calls" % reps}
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle legs
 # ---------------------------------------------------------------------------
@@ -209,8 +283,8 @@ def run_reference(args, rank, world):
             "ms_per_step": 1000 * tot / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config(wl, {"sample": sample}),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": dict({"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                  "sample": sample}, **_host_cpu()),
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -309,6 +383,17 @@ def run_ours(args, rank, world, local_rank):
 
     if rank != 0:
         return
+    # per-run report (untimed): zero shares, effective bpw, safeguard count
+    reports = []
+    for wl, A, w, out in zip(wls, As, Ws, outs):
+        stats = None
+        if wl.block <= 1:
+            _, tr, _ = X.decompose_traced(A, wl.mu, wl.tau, wl.iters, [], w=w)
+            stats = tr.stats.cpu().numpy()
+        reports.append(_factor_report(out, stats))
+    smem_gbs, l2_gbs = _onchip_peaks(X, dev)
+    peak0, _ = _peaks()
+    apply_m = _apply_measure(X, outs[0], dev, flush, peak0) if wls[0].m <= 16384 else None
     # roofline: algorithmic residual traffic, 4 m n (2I + 2) bytes per component
     # (sequential) or per block of components (block-ALS)
     alg_bytes = 0.0
@@ -323,6 +408,13 @@ def run_ours(args, rank, world, local_rank):
     traffic = _profiled_traffic(kernel, wls[0].name) if len(wls) == 1 else None
     roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
             "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+            "onchip": {"resource": "smem" if sequential else "l2",
+                       "peak": smem_gbs if sequential else l2_gbs, "unit": "GB/s",
+                       "frac": achieved / (smem_gbs if sequential else l2_gbs),
+                       "smem_peak_gbs": smem_gbs, "l2_peak_gbs": l2_gbs,
+                       "probe": "externd_probe_read_bandwidth in this run: every SM streams "
+                                "192 KB of its shared memory / a 26 MiB L2-resident buffer, "
+                                "128-bit loads, best of 3"},
             "kernel": kernel, "alg_bytes_per_launch": alg_bytes if sequential else None,
             "alg_bytes_per_step": alg_bytes,
             "note": ("residual R is resident in shared memory across the grid; algorithmic "
@@ -341,8 +433,14 @@ def run_ours(args, rank, world, local_rank):
                 "achieved_gbs": achieved})
     if len(wls) == 1:
         cfg["energy_preserved_pct"] = 100.0 * energies[0]
+        cfg.update(reports[0])
+        if sequential:
+            # the rank this matrix needs for Q4_K's per-matrix energy (99.4%,
+            # Pith review), read off the run's energy trace on the device
+            cfg["rank_for_99.4pct_energy"] = X.rank_for_energy(outs[0].energy, 0.994)
     else:
         cfg["energy_preserved_pct"] = {wl.name: 100.0 * e for wl, e in zip(wls, energies)}
+        cfg["factors"] = {wl.name: r for wl, r in zip(wls, reports)}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": sum(step_ms) / args.steps, "higher_is_better": True,
@@ -351,15 +449,17 @@ def run_ours(args, rank, world, local_rank):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * sum(_launches_per_decomposition(wl) for wl in wls),
+            "ternary_apply": apply_m,
             "clocks": clk.summary(),
             "step_ms": step_ms}
     if world == 1 and not args.no_cpu_baseline:
         wl0 = wls[0]
         ncomp = _env_int("EXTERND_CPU_COMPONENTS", 96 if wl0.block <= 1 else 2 * wl0.block)
         t = _oracle_prefix(wl0, ncomp)
-        line["cpu_baseline"] = {"value": ncomp / t, "unit": UNIT, "cores": 1, "kind": "oracle",
-                                "sample": f"first {ncomp} of {wl0.k} components of {wl0.name}, "
-                                          f"free-running oracle from A, one thread"}
+        line["cpu_baseline"] = dict({"value": ncomp / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                     "sample": f"first {ncomp} of {wl0.k} components of "
+                                               f"{wl0.name}, free-running oracle from A, one "
+                                               f"thread"}, **_host_cpu())
     print(json.dumps(line), flush=True)
 
 
@@ -375,6 +475,21 @@ def run_case(args):
     elif args.case == "mlp9728_3blocks":
         wl = W.config_mlp9728(64)
         mu, block = 3 * 64 / min(wl.m, wl.n), 64
+    elif args.case == "apply_attn2560":
+        # the inference kernel on the benchmark matrix's factors (mu = 3): the
+        # decomposition, then three one-vector calls
+        wl = W.config_attn2560()
+        A = torch.from_numpy(wl.a).cuda()
+        f = X.decompose(A, wl.mu, wl.tau, wl.iters)
+        x = torch.randn(1, wl.n, device="cuda")
+        for _ in range(3):
+            y = X.apply(f, x)
+        torch.cuda.synchronize()
+        st = X.sync_status()
+        print(json.dumps({"case": args.case, "k": f.k, "y0": float(y[0, 0]), "status": st}))
+        if st != X.OK:
+            raise SystemExit(1)
+        return
     else:
         raise SystemExit(f"unknown case {args.case}")
     A = torch.from_numpy(wl.a).cuda()
@@ -395,7 +510,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=WORKLOADS, default="attn2560")
-    ap.add_argument("--case", choices=("attn2560_k64", "mlp9728_3blocks"), default=None)
+    ap.add_argument("--case", choices=("attn2560_k64", "mlp9728_3blocks", "apply_attn2560"),
+                    default=None)
     args = ap.parse_args()
     if args.case:
         run_case(args)

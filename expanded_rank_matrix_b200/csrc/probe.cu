@@ -1,0 +1,110 @@
+// Read-bandwidth probes for the on-chip rooflines: shared memory (every SM
+// streams its own shared memory) and L2 (every SM streams an L2-resident
+// buffer).  The sequential kernel keeps the residual in shared memory and
+// the block path's operands mostly in L2, so their kernels are judged
+// against these rates as well as against HBM.
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/externd.h"
+
+namespace {
+
+constexpr int kProbeThreads = 512;
+constexpr int kProbeUnroll = 8;
+
+__global__ void __launch_bounds__(kProbeThreads, 1) smem_probe(int bytes, int reps,
+                                                                 unsigned long long* sink) {
+  extern __shared__ __align__(16) float4 sp[];
+  const int n4 = bytes / 16;
+  for (int e = threadIdx.x; e < n4; e += kProbeThreads)
+    sp[e] = make_float4((float)e, 1.f, 2.f, 3.f);
+  __syncthreads();
+  const int per = kProbeThreads * kProbeUnroll, iters = n4 / per;
+  float acc[kProbeUnroll];
+#pragma unroll
+  for (int u = 0; u < kProbeUnroll; ++u) acc[u] = 0.f;
+  for (int r = 0; r < reps; ++r) {
+    for (int it = 0; it < iters; ++it) {
+      const float4* q = sp + it * per + threadIdx.x;
+      float4 x[kProbeUnroll];
+#pragma unroll
+      for (int u = 0; u < kProbeUnroll; ++u) x[u] = q[u * kProbeThreads];
+#pragma unroll
+      for (int u = 0; u < kProbeUnroll; ++u) acc[u] += (x[u].x + x[u].y) + (x[u].z + x[u].w);
+    }
+    __syncthreads();
+  }
+  float s = 0.f;
+#pragma unroll
+  for (int u = 0; u < kProbeUnroll; ++u) s += acc[u];
+  if (s == 1.2345f) sink[blockIdx.x] = 1ull;  // keeps the loads
+}
+
+__global__ void __launch_bounds__(kProbeThreads) l2_probe(const float4* __restrict__ buf,
+                                                          long long n4, int reps,
+                                                          unsigned long long* sink) {
+  // the reps passes form one long sequence of n4 * reps loads, so every
+  // thread keeps kProbeUnroll loads in flight however small the buffer
+  const long long stride = (long long)gridDim.x * kProbeThreads, total = n4 * reps;
+  float acc = 0.f;
+  long long e = (long long)blockIdx.x * kProbeThreads + threadIdx.x;
+  for (; e + (kProbeUnroll - 1) * stride < total; e += kProbeUnroll * stride) {
+    float4 x[kProbeUnroll];
+#pragma unroll
+    for (int u = 0; u < kProbeUnroll; ++u) x[u] = __ldcg(buf + (e + u * stride) % n4);
+#pragma unroll
+    for (int u = 0; u < kProbeUnroll; ++u) acc += (x[u].x + x[u].y) + (x[u].z + x[u].w);
+  }
+  for (; e < total; e += stride) {
+    const float4 x = __ldcg(buf + e % n4);
+    acc += (x.x + x.y) + (x.z + x.w);
+  }
+  if (acc == 1.2345f) sink[blockIdx.x] = 1ull;
+}
+
+}  // namespace
+
+extern "C" int externd_probe_read_bandwidth(int kind, const void* buf, int64_t bytes, int reps,
+                                            int64_t* bytes_read, externd_stream_t stream) {
+  if (reps < 1 || !bytes_read) return EXTERND_ERR_INVALID_ARG;
+  int dev = 0, nsm = 0, optin = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return EXTERND_ERR_CUDA;
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned long long* sink = nullptr;
+  if (cudaMallocAsync(&sink, sizeof(unsigned long long) * (size_t)nsm * 4, st) != cudaSuccess) {
+    cudaGetLastError();
+    return EXTERND_ERR_OOM;
+  }
+  int rc = EXTERND_OK;
+  if (kind == EXTERND_PROBE_SMEM) {
+    // the largest multiple of one pass (threads x unroll x 16 bytes) that fits
+    const int pass = kProbeThreads * kProbeUnroll * 16;
+    const int sbytes = (optin - 1024) / pass * pass;
+    if (sbytes < pass ||
+        cudaFuncSetAttribute(smem_probe, cudaFuncAttributeMaxDynamicSharedMemorySize, sbytes) !=
+            cudaSuccess) {
+      rc = EXTERND_ERR_CUDA;
+    } else {
+      smem_probe<<<nsm, kProbeThreads, sbytes, st>>>(sbytes, reps, sink);
+      *bytes_read = (int64_t)nsm * sbytes * reps;
+    }
+  } else if (kind == EXTERND_PROBE_L2) {
+    if (!buf || bytes < 16 || ((uintptr_t)buf & 15u)) {
+      rc = EXTERND_ERR_INVALID_ARG;
+    } else {
+      const long long n4 = bytes / 16;
+      l2_probe<<<nsm * 4, kProbeThreads, 0, st>>>((const float4*)buf, n4, reps, sink);
+      *bytes_read = (int64_t)n4 * 16 * reps;
+    }
+  } else {
+    rc = EXTERND_ERR_INVALID_ARG;
+  }
+  if (rc == EXTERND_OK && cudaGetLastError() != cudaSuccess) rc = EXTERND_ERR_CUDA;
+  if (cudaFreeAsync(sink, st) != cudaSuccess && rc == EXTERND_OK) rc = EXTERND_ERR_CUDA;
+  return rc;
+}

@@ -35,7 +35,7 @@ MAX_SWEEPS = 64
 EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_ex", "externd_decompose_traced",
            "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc",
            "externd_decompose_block_traced", "externd_rank_for_energy",
-           "externd_ternary_apply")
+           "externd_ternary_apply", "externd_probe_read_bandwidth")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -83,6 +83,9 @@ def load(path: str = LIB_PATH):
     L.externd_rank_for_energy.restype = ctypes.c_int
     L.externd_ternary_apply.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _i64, _vp, _vp]
     L.externd_ternary_apply.restype = ctypes.c_int
+    L.externd_probe_read_bandwidth.argtypes = [ctypes.c_int, _vp, _i64, ctypes.c_int,
+                                               ctypes.POINTER(ctypes.c_int64), _vp]
+    L.externd_probe_read_bandwidth.restype = ctypes.c_int
     L.externd_sync_status.argtypes = [_vp]
     L.externd_sync_status.restype = ctypes.c_int
     _lib = L
@@ -292,6 +295,28 @@ def apply(f: Factors, X: torch.Tensor, stream: Optional[torch.cuda.Stream] = Non
     Y = torch.empty((X2.shape[0], f.m), dtype=torch.float32, device=X.device)
     apply_into(f, X2, Y, stream)
     return Y.reshape(*X.shape[:-1], f.m)
+
+
+PROBE_SMEM = 0
+PROBE_L2 = 1
+
+
+def probe_read_bandwidth(kind: int, reps: int, buf: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None) -> float:
+    """Measured read bandwidth (bytes/s) of shared memory (PROBE_SMEM, every
+    SM) or of an L2-resident buffer (PROBE_L2), timed with CUDA events."""
+    out = ctypes.c_int64(0)
+    s = stream if stream is not None else torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    nbytes = 0 if buf is None else buf.numel() * buf.element_size()
+    ev0.record(s)
+    rc = load().externd_probe_read_bandwidth(kind, _ptr(buf) if buf is not None else None, nbytes,
+                                             reps, ctypes.byref(out), _stream(s))
+    ev1.record(s)
+    if rc != OK:
+        raise ExterndError(rc, "externd_probe_read_bandwidth")
+    ev1.synchronize()
+    return out.value / (ev0.elapsed_time(ev1) / 1000.0)
 
 
 def sync_status(stream: Optional[torch.cuda.Stream] = None) -> int:

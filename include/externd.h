@@ -235,8 +235,9 @@ int externd_reconstruct(const uint32_t* packed_B, const uint32_t* packed_C, cons
  *   X        [nb][n] fp32 (device, in): nb input vectors, row-major.
  *   nb       1 .. 65536 vectors (processed two at a time).
  *   Y        [nb][m] fp32 (device, out).
- * Scratch (k + SMs * m) * 2 floats, stream-ordered on `stream` like
- * externd_decompose's.  One cooperative launch per two vectors (every CTA
+ * Scratch: SMs * m * 2 floats, stream-ordered on `stream` from a memory pool
+ * the library owns on each device, which keeps that memory mapped between
+ * calls (until the process exits).  One cooperative launch per two vectors (every CTA
  * resident; its two grid barriers are bounded waits that raise
  * EXTERND_ERR_TIMEOUT in the status word if they ever run out).  Returns
  * EXTERND_OK, EXTERND_ERR_INVALID_ARG, EXTERND_ERR_OOM, EXTERND_ERR_NO_COOP
@@ -305,6 +306,22 @@ int externd_decompose_noalloc(const float* A, int64_t m, int64_t n, float mu, fl
  */
 int externd_rank_for_energy(const double* energy_trace, int64_t k, double target, int64_t* rank,
                             externd_stream_t stream);
+
+/*
+ * externd_probe_read_bandwidth -- a read-bandwidth probe for the on-chip
+ * rooflines (measurement, not part of the method).  kind
+ * EXTERND_PROBE_SMEM: one CTA per SM streams its own shared memory (about
+ * 220 KB) `reps` times with 128-bit loads; buf and bytes are ignored.
+ * EXTERND_PROBE_L2: every SM streams the device buffer `buf` (`bytes` long,
+ * 16-byte aligned; size it well below the L2 so it stays resident) `reps`
+ * times with 128-bit L2 loads.  *bytes_read (host) receives the bytes the
+ * launch reads; time it with events on `stream`.  Returns EXTERND_OK,
+ * EXTERND_ERR_INVALID_ARG, EXTERND_ERR_OOM or EXTERND_ERR_CUDA.
+ */
+#define EXTERND_PROBE_SMEM 0
+#define EXTERND_PROBE_L2 1
+int externd_probe_read_bandwidth(int kind, const void* buf, int64_t bytes, int reps,
+                                 int64_t* bytes_read, externd_stream_t stream);
 
 /*
  * externd_sync_status -- synchronises `stream`, then returns and clears the
