@@ -70,6 +70,9 @@ __global__ void __launch_bounds__(kProbeThreads) l2_probe(const float4* __restri
 extern "C" int externd_probe_read_bandwidth(int kind, const void* buf, int64_t bytes, int reps,
                                             int64_t* bytes_read, externd_stream_t stream) {
   if (reps < 1 || !bytes_read) return EXTERND_ERR_INVALID_ARG;
+  if (kind != EXTERND_PROBE_SMEM && kind != EXTERND_PROBE_L2) return EXTERND_ERR_INVALID_ARG;
+  if (kind == EXTERND_PROBE_L2 && (!buf || bytes < 16 || ((uintptr_t)buf & 15u)))
+    return EXTERND_ERR_INVALID_ARG;
   int dev = 0, nsm = 0, optin = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return EXTERND_ERR_CUDA;
   cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);

@@ -152,3 +152,17 @@ def test_ternary_apply_argument_checks(lib):
                                    nul) == X.ERR_INVALID_ARG  # more rows than one launch covers
     mis = ctypes.c_void_p((1 << 20) + 2)
     assert L.externd_ternary_apply(fake, fake, fake, 8, 8, 4, mis, 1, fake, nul) == X.ERR_INVALID_ARG
+
+
+def test_probe_argument_checks(lib):
+    L = lib
+    out = ctypes.c_int64(0)
+    fake = ctypes.c_void_p(1 << 20)
+    assert L.externd_probe_read_bandwidth(7, None, 0, 1, ctypes.byref(out), None) == X.ERR_INVALID_ARG
+    assert L.externd_probe_read_bandwidth(X.PROBE_SMEM, None, 0, 0, ctypes.byref(out),
+                                          None) == X.ERR_INVALID_ARG
+    assert L.externd_probe_read_bandwidth(X.PROBE_L2, None, 1 << 20, 1, ctypes.byref(out),
+                                          None) == X.ERR_INVALID_ARG
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    assert L.externd_probe_read_bandwidth(X.PROBE_L2, mis, 1 << 20, 1, ctypes.byref(out),
+                                          None) == X.ERR_INVALID_ARG
