@@ -8,7 +8,11 @@
 
 namespace externd {
 
-constexpr int kThreads = 512;  // threads per CTA of the persistent kernels
+// threads per CTA of the persistent sequential kernel: twelve warps, so the
+// kernel may hold 168 registers per thread (at sixteen warps the 128-register
+// cap spills its loop state, and with the residual filling shared memory the
+// spills miss L1)
+constexpr int kThreads = 384;
 constexpr int kWarps = kThreads / 32;
 constexpr long long kDefaultWaitBudget = 2000000000LL;  // SM cycles, about 1 s
 

@@ -726,8 +726,11 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     float* x_bs = (float*)(xu + 3 * a.NC);
     float* x_bv = (float*)(xu + 4 * a.NC);
     double* rsa = (double*)zred;  // [NC][CS] slice sums of squares (one-round path)
-    const bool one_round = !with_row || (a.NC <= 16 && TC + a.NC + a.NC * CS <= kThreads &&
+    const bool one_round = !with_row || (a.NC <= 16 && TC + a.NC <= kThreads &&
                                          2 * a.NC * CS <= L.zred_floats);
+    // the CTAs' slice statistics: a thread each when the block has enough
+    // threads, else the record threads fetch their cluster's as well
+    const bool rsa_own = TC + a.NC + a.NC * CS <= kThreads;
     const long long cstride = (long long)CS * a.recw;
     const int rbase = (with_row && one_round) ? TC : 0;  // first thread of the record range
     uint32_t slice[16];
@@ -742,7 +745,14 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       x_bv[cc] = u2f(p[5]);
       x_r2[cc] = u2d(p[6], p[7]);
       x_bad[cc] = p[8];
-    } else if (with_row && one_round && tid >= TC + a.NC && tid < TC + a.NC + a.NC * CS) {
+      if (with_row && one_round && !rsa_own)
+        for (int qq = 0; qq < CS; ++qq) {
+          uint32_t p2[2];
+          xw_wait_n<2>(rec(s, cc, qq) + TCp, 1, 2, ep, p2, ab, a.budget, a.abort_word);
+          rsa[cc * CS + qq] = u2d(p2[0], p2[1]);
+        }
+    } else if (with_row && one_round && rsa_own && tid >= TC + a.NC &&
+               tid < TC + a.NC + a.NC * CS) {
       const int t = tid - TC - a.NC, cc = t / CS, qq = t - cc * CS;
       uint32_t p[2];
       xw_wait_n<2>(rec(s, cc, qq) + TCp, 1, 2, ep, p, ab, a.budget, a.abort_word);
@@ -955,7 +965,7 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
         if (K == 4) y_rows<4, 2>(tsb, TCp, TRs, g, qy0, qy1, vw4, ps);
         else if (K == 3) y_rows<3, 3>(tsb, TCp, TRs, g, qy0, qy1, vw4, ps);
         else if (K == 2) y_rows<2, 4>(tsb, TCp, TRs, g, qy0, qy1, vw4, ps);
-        else y_rows<1, 6>(tsb, TCp, TRs, g, qy0, qy1, vw4, ps);
+        else y_rows<1, 12>(tsb, TCp, TRs, g, qy0, qy1, vw4, ps);
       }
       if (HYB && gr0 < gr1) {
         float4 vr[NQL];
@@ -1124,6 +1134,32 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       if (rgz < RGz) {
         float4 za = make_float4(0.f, 0.f, 0.f, 0.f), zb = za;
         int t2 = rgz;
+        for (; t2 + 3 * RGz < nnz_c; t2 += 4 * RGz) {
+          const int e0 = rlist[t2], e1 = rlist[t2 + RGz], e2 = rlist[t2 + 2 * RGz],
+                    e3 = rlist[t2 + 3 * RGz];
+          const float4 x0 = ld4(e0 >= 0 ? e0 : ~e0, qz);
+          const float4 x1 = ld4(e1 >= 0 ? e1 : ~e1, qz);
+          const float4 x2 = ld4(e2 >= 0 ? e2 : ~e2, qz);
+          const float4 x3 = ld4(e3 >= 0 ? e3 : ~e3, qz);
+          const float s0 = e0 >= 0 ? 1.f : -1.f, s1 = e1 >= 0 ? 1.f : -1.f;
+          const float s2 = e2 >= 0 ? 1.f : -1.f, s3 = e3 >= 0 ? 1.f : -1.f;
+          za.x = fmaf(s0, x0.x, za.x);
+          za.y = fmaf(s0, x0.y, za.y);
+          za.z = fmaf(s0, x0.z, za.z);
+          za.w = fmaf(s0, x0.w, za.w);
+          zb.x = fmaf(s1, x1.x, zb.x);
+          zb.y = fmaf(s1, x1.y, zb.y);
+          zb.z = fmaf(s1, x1.z, zb.z);
+          zb.w = fmaf(s1, x1.w, zb.w);
+          za.x = fmaf(s2, x2.x, za.x);
+          za.y = fmaf(s2, x2.y, za.y);
+          za.z = fmaf(s2, x2.z, za.z);
+          za.w = fmaf(s2, x2.w, za.w);
+          zb.x = fmaf(s3, x3.x, zb.x);
+          zb.y = fmaf(s3, x3.y, zb.y);
+          zb.z = fmaf(s3, x3.z, zb.z);
+          zb.w = fmaf(s3, x3.w, zb.w);
+        }
         for (; t2 + RGz < nnz_c; t2 += 2 * RGz) {
           const int e0 = rlist[t2], e1 = rlist[t2 + RGz];
           const float4 x0 = ld4(e0 >= 0 ? e0 : ~e0, qz);
