@@ -78,8 +78,9 @@ int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float m
                                    uint32_t* packed_B,
                                    uint32_t* packed_C, float* D, double* energy_trace,
                                    int64_t ntrace, const int64_t* trace_block, uint64_t* trace_uv,
-                                   int32_t* trace_rows, externd_stream_t stream) {
-  if (block < 2) return EXTERND_ERR_INVALID_ARG;
+                                   int32_t* trace_rows, int64_t wait_budget,
+                                   externd_stream_t stream) {
+  if (block < 2 || wait_budget < 0) return EXTERND_ERR_INVALID_ARG;
   if (ntrace < 0 || (ntrace > 0 && (!trace_block || !trace_uv || !trace_rows)))
     return EXTERND_ERR_INVALID_ARG;
   if (!A || !packed_B || !packed_C || !D || !energy_trace) return EXTERND_ERR_INVALID_ARG;
@@ -97,7 +98,7 @@ int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float m
   b.A = A; b.m = m; b.n = n; b.k = k; b.tau = tau; b.iters = iters; b.w = w; b.block = block;
   b.packed_B = packed_B; b.packed_C = packed_C; b.D = D; b.energy = energy_trace;
   b.ntrace = ntrace; b.trace_block = trace_block; b.trace_uv = trace_uv; b.trace_rows = trace_rows;
-  b.flags = flags;
+  b.flags = flags; b.wait_budget = wait_budget;
   return externd::block_decompose(b, (cudaStream_t)stream);
 }
 
@@ -137,6 +138,12 @@ int externd_ternary_apply(const uint32_t* packed_B, const uint32_t* packed_C, co
   if (nb < 1 || nb > 65536 || nb * (m > n ? m : n) >= ((int64_t)1 << 31))
     return EXTERND_ERR_INVALID_ARG;
   return externd::ternary_apply(packed_B, packed_C, D, m, n, k, X, nb, Y, (cudaStream_t)stream);
+}
+
+int externd_release_cache(void) {
+  const int a = externd::block_release_graphs();
+  const int b = externd::apply_trim_pools();
+  return a != EXTERND_OK ? a : b;
 }
 
 int externd_sync_status(externd_stream_t stream) {

@@ -264,11 +264,13 @@ int launch_apply(ApArgs a, int G, size_t smem, cudaStream_t st) {
 // device, which keeps its memory mapped between calls (the default pool
 // returns freed memory at every synchronisation, and mapping it again costs
 // more than the kernel).
+std::mutex g_pool_mu;
+cudaMemPool_t g_pools[64] = {};
+
 cudaMemPool_t apply_pool(int dev) {
-  static std::mutex mu;
-  static cudaMemPool_t pools[64] = {};
+  cudaMemPool_t* const pools = g_pools;
   if (dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lk(mu);
+  std::lock_guard<std::mutex> lk(g_pool_mu);
   if (!pools[dev]) {
     cudaMemPoolProps props = {};
     props.allocType = cudaMemAllocationTypePinned;
@@ -287,6 +289,18 @@ cudaMemPool_t apply_pool(int dev) {
 }
 
 }  // namespace
+
+// Returns the memory the pools hold beyond what queued calls still use.
+int apply_trim_pools() {
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  int rc = EXTERND_OK;
+  for (cudaMemPool_t p : g_pools)
+    if (p && cudaMemPoolTrimTo(p, 0) != cudaSuccess) {
+      cudaGetLastError();
+      rc = EXTERND_ERR_CUDA;
+    }
+  return rc;
+}
 
 int ternary_apply(const uint32_t* pB, const uint32_t* pC, const float* D, int64_t m, int64_t n,
                   int64_t k, const float* X, int64_t nb, float* Y, cudaStream_t st) {

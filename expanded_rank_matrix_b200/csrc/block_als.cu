@@ -1116,7 +1116,7 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
       inv_kernel<<<1, 256, 0, side>>>(GV, bb, SV);
       cudaEventRecord(ev_join, side);
       tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, sk ? &planP : nullptr, klenP, splitP,
-                     Pp, st);
+                     Pp, h.wait_budget, st);
       cudaStreamWaitEvent(st, ev_join, 0);
       tgtP<<<tgtU, 256, kTgtSmem, st>>>(Pp, splitP, m, bb, SV, tau, T, Cs, tick, thr, nullptr, sk,
                                          planP.C, planP.U, planP.G, planP.S, stat, nullptr);
@@ -1126,7 +1126,8 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
       gram_kernel<<<gblocks, gthreads, 0, side>>>(pB, Wm, bb, nullptr, GU);
       inv_kernel<<<1, 256, 0, side>>>(GU, bb, SU);
       cudaEventRecord(ev_join, side);
-      tc_contract_rtu(R, m, n, Um, Us, BopU, bb, sk ? &planQ : nullptr, klenQ, splitQ, Qp, st);
+      tc_contract_rtu(R, m, n, Um, Us, BopU, bb, sk ? &planQ : nullptr, klenQ, splitQ, Qp,
+                      h.wait_budget, st);
       cudaStreamWaitEvent(st, ev_join, 0);
       tgtQ<<<tgtV, 256, kTgtSmem, st>>>(Qp, splitQ, n, bb, SU, tau, T, Cs, tick, thr,
                                          it == h.iters - 1 ? Qs : nullptr, sk, planQ.C, planQ.U,
@@ -1167,7 +1168,8 @@ struct GraphKey {
     return h.A == o.h.A && h.m == o.h.m && h.n == o.h.n && h.k == o.h.k && h.tau == o.h.tau &&
            h.iters == o.h.iters && h.w == o.h.w && h.block == o.h.block &&
            h.flags == o.h.flags && h.packed_B == o.h.packed_B && h.packed_C == o.h.packed_C &&
-           h.D == o.h.D && h.energy == o.h.energy && dev == o.dev && no_tma == o.no_tma;
+           h.D == o.h.D && h.energy == o.h.energy && h.wait_budget == o.h.wait_budget &&
+           dev == o.dev && no_tma == o.no_tma;
   }
 };
 
@@ -1289,11 +1291,34 @@ int block_decompose(const BlockHostArgs& h, cudaStream_t st) {
   g.key = key;
   if (capture(g, h) != EXTERND_OK) return enqueue_direct(h, st);
   if (g_graphs.size() >= kGraphSlots) {
+    const int edev = g_graphs.front().key.dev;
     release(g_graphs.front());
     g_graphs.erase(g_graphs.begin());
+    // the evicted graph's workspace goes back to the device once it is idle
+    int cur = 0;
+    if (cudaGetDevice(&cur) == cudaSuccess && cur == edev) cudaDeviceGraphMemTrim(edev);
+    cudaGetLastError();
   }
   g_graphs.push_back(g);
   return replay(g_graphs.back(), st);
+}
+
+int block_release_graphs() {
+  std::lock_guard<std::mutex> lock(g_graph_mu);
+  bool devs[64] = {};
+  for (GraphSlot& g : g_graphs) {
+    if (g.key.dev >= 0 && g.key.dev < 64) devs[g.key.dev] = true;
+    release(g);
+  }
+  g_graphs.clear();
+  g_seen.clear();
+  int rc = EXTERND_OK;
+  for (int d = 0; d < 64; ++d)
+    if (devs[d] && cudaDeviceGraphMemTrim(d) != cudaSuccess) {
+      cudaGetLastError();
+      rc = EXTERND_ERR_CUDA;
+    }
+  return rc;
 }
 
 }  // namespace externd

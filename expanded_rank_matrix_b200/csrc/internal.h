@@ -45,6 +45,7 @@ struct BlockHostArgs {
   uint64_t* trace_uv;          // device: per traced block, V0 then U_t, V_t masks
   int32_t* trace_rows;         // device: per traced block, the start rows
   unsigned flags;              // EXTERND_TSTAT_MEAN_ABS | EXTERND_VSTEP_NAIVE
+  int64_t wait_budget;         // SM cycles for the contractions' waits (0: default)
 };
 
 int seq_decompose(const SeqHostArgs& h, cudaStream_t st);
@@ -70,10 +71,12 @@ bool tc_contract_tma_ok(int n);  // n % 4 == 0 and the tensor-map encoder is ava
 int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
                    const unsigned long long* Vs, const unsigned char* Bop, const float* w,
                    const float* wpad, int bb, const TcPlan* p, int klen, int splits, float* Pp,
-                   cudaStream_t st);
+                   long long budget, cudaStream_t st);
 int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
                     const unsigned long long* Us, const unsigned char* Bop, int bb, const TcPlan* p,
-                    int klen, int splits, float* Qp, cudaStream_t st);
+                    int klen, int splits, float* Qp, long long budget, cudaStream_t st);
+int block_release_graphs();
+int apply_trim_pools();
 int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
                                cudaStream_t st);
 

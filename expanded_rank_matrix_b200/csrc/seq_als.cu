@@ -171,12 +171,24 @@ struct SeqPlan {
   size_t smem = 0;
 };
 
+// Bytes of caller-provided scratch a plan needs when nothing is allocated:
+// the three exchange rings, then the abort word on its own 256-byte line.
+static size_t fixed_scratch_bytes(int NC, int CS, int TCp) {
+  const size_t xbytes = sizeof(uint64_t) * 3 * (size_t)NC * CS * (TCp + 16);
+  return ((xbytes + 255) & ~(size_t)255) + 256;
+}
+
 // Chooses cluster size, cluster count and how many rows of each CTA's tile
 // stay in shared memory (the rest stream from global memory).  Candidates
 // must be co-resident (occupancy query).  The estimated cost per half-step
 // -- tile words read per CTA, global rows weighted 4x, plus the cross-cluster
-// words each CTA polls -- is minimised.
-static cudaError_t plan_seq(int m, int n, bool weighted, cudaStream_t st, SeqPlan* out) {
+// words each CTA polls -- is minimised.  With scratch_limit > 0 only plans
+// that keep the whole residual in shared memory and whose exchange rings fit
+// in scratch_limit bytes are candidates; the best of all plans is among them
+// whenever it qualifies, so such a call takes the same plan as an
+// unrestricted one in that case.
+static cudaError_t plan_seq(int m, int n, bool weighted, cudaStream_t st, SeqPlan* out,
+                            size_t scratch_limit = 0) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -225,6 +237,9 @@ static cudaError_t plan_seq(int m, int n, bool weighted, cudaStream_t st, SeqPla
         break;
       }
       if (maxc >= nc) {
+        if (scratch_limit > 0 &&
+            (SR < TRmax || fixed_scratch_bytes(nc, CS, TCp) > scratch_limit))
+          break;  // fewer clusters only lengthen the tile rows
         const double tile_w = (double)SR * TCp + 4.0 * (double)(TRmax - SR) * TCp;
         const double cost = tile_w + 8.0 * nc * TCp;
         if (cost < best_cost) {
@@ -349,17 +364,16 @@ int seq_decompose(const SeqHostArgs& h, cudaStream_t st) {
 int seq_decompose_with_scratch(const SeqHostArgs& h, void* scratch, size_t scratch_bytes,
                                cudaStream_t st) {
   if (h.sweeps != 0) return EXTERND_ERR_INVALID_ARG;
+  if (scratch_bytes < 256) return EXTERND_ERR_SCRATCH_LIMIT;
   SeqPlan pl;
-  cudaError_t e = plan_seq((int)h.m, (int)h.n, h.w != nullptr, st, &pl);
-  if (e == cudaErrorNotSupported) return EXTERND_ERR_NO_COOP;
+  cudaError_t e = plan_seq((int)h.m, (int)h.n, h.w != nullptr, st, &pl, scratch_bytes);
+  if (e == cudaErrorNotSupported) return EXTERND_ERR_SCRATCH_LIMIT;
   if (e != cudaSuccess) return EXTERND_ERR_CUDA;
-  if (pl.SR < pl.TRmax) return EXTERND_ERR_SCRATCH_LIMIT;
   const int recw = pl.TCp + 16;
   const long long slot_words = (long long)pl.NC * pl.CS * recw;
-  const size_t xbytes = sizeof(uint64_t) * 3 * (size_t)slot_words;
-  const size_t abort_off = (xbytes + 255) & ~(size_t)255;
-  const size_t need = abort_off + 256;
-  if (need > scratch_bytes) return EXTERND_ERR_SCRATCH_LIMIT;
+  const size_t need = fixed_scratch_bytes(pl.NC, pl.CS, pl.TCp);
+  const size_t abort_off = need - 256;
+  if (pl.SR < pl.TRmax || need > scratch_bytes) return EXTERND_ERR_SCRATCH_LIMIT;
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return EXTERND_ERR_CUDA;
   if (clear_outputs(h, st) != cudaSuccess) return EXTERND_ERR_CUDA;
   SeqArgs a = {};

@@ -9,14 +9,29 @@
 // product the tensor core forms is exact and only its fp32 accumulation rounds
 // -- the same class of error as an fp32 dot product on the CUDA cores.
 //
-// Per CTA: one 128 x 64 fp32 accumulator in tensor memory; the K range of the
-// CTA's split is walked in chunks of 32, double buffered in shared memory:
-// all threads convert a chunk into the canonical no-swizzle UMMA layouts while
-// the tensor core runs the 3 x 2 MMAs (3 parts x K/16 steps) of the previous
-// chunk, issued by one thread; tcgen05.commit on a per-stage mbarrier tells when a stage may be
-// refilled.  Every mbarrier wait is bounded; a wait that runs out records
-// EXTERND_ERR_TIMEOUT, the CTA stops issuing, drains (bounded) and frees its
-// tensor memory.  Outputs are split-K partials Xp[split][row][64].
+// Two kernels compute these contractions; tc_contract_rv / tc_contract_rtu
+// choose between them.
+//
+// contract_tma_kernel (the usual path: rows of R 16-byte aligned, i.e.
+// n % 4 == 0): persistent, one CTA per SM, stream-K over units of (128-row
+// tile, 32-wide K chunk).  A producer thread copies fp32 chunks of R with TMA
+// (and the ternary B chunks with bulk copies) into an 8-deep shared-memory
+// ring; converter warps split each chunk into its bf16 parts straight into
+// tensor memory; one thread issues the MMAs into one of two alternating
+// 128 x 64 fp32 accumulators in tensor memory; epilogue warps read a finished
+// accumulator out (tcgen05.ld) into the tile's stream-K partials
+// Xp[(t S + slot) 128 + row][64] while the next segment streams.
+//
+// contract_kernel (the other case: n % 4 != 0, or EXTERND_CONTRACT_NO_TMA=1):
+// one CTA per (128-row tile, K split); every thread loads and converts a
+// chunk into the canonical no-swizzle UMMA layouts in shared memory, double
+// buffered, while one thread issues the previous chunk's 3 x 2 MMAs (3 parts
+// x K/16 steps); tcgen05.commit on a per-stage mbarrier tells when a stage
+// may be refilled.  Outputs are split-K partials Xp[split][row][64].
+//
+// In both, every mbarrier wait is bounded; a wait that runs out records
+// EXTERND_ERR_TIMEOUT, the CTA stops issuing, waits (bounded) for its own
+// copies and MMAs in flight and frees its tensor memory.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -455,16 +470,17 @@ __device__ __forceinline__ void umma_ts_bf16(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
-// Bounded wait that also gives up once another thread of the CTA has
-// recorded a timeout in *abort.
+// Bounded wait (budget in SM cycles) that also gives up once another thread
+// of the CTA has recorded a timeout in *abort.  The waits for the CTA's own
+// copies and MMAs before it exits use mbar_wait (kWaitBudget) instead.
 __device__ __forceinline__ bool mbar_wait_ab(uint32_t addr, uint32_t parity,
-                                             volatile int* abort) {
+                                             volatile int* abort, long long budget) {
   if (mbar_test(addr, parity)) return true;
   const long long t0 = clock64();
   unsigned spins = 0;
   while (!mbar_test(addr, parity)) {
     if (((++spins) & 15u) == 0u && *abort) return false;
-    if (clock64() - t0 > kWaitBudget) {
+    if (clock64() - t0 > budget) {
       *abort = 1;
       return false;
     }
@@ -492,7 +508,7 @@ template <int MODE>
 __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
     const __grid_constant__ CUtensorMap tmap, int m, int n, const unsigned char* __restrict__ Bop,
     const float* __restrict__ wpad, int bb, int C, long long U, int S, float* __restrict__ Xp,
-    int* __restrict__ status) {
+    int* __restrict__ status, long long budget) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* ring = (unsigned char*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) PipeBars bars;
@@ -540,7 +556,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
         const int s = i % kS32;
         // stage s (fp32 tile, B, A in tensor memory) is free once the MMAs
         // of chunk i - kS32 have completed
-        if (i >= kS32 && !mbar_wait_ab(smem_u32(&bars.aempty[s]), ((i / kS32) + 1) & 1, ab))
+        if (i >= kS32 && !mbar_wait_ab(smem_u32(&bars.aempty[s]), ((i / kS32) + 1) & 1, ab, budget))
           break;
         const int kk = c * kKc;
         const uint32_t fb = smem_u32(&bars.full[s]);
@@ -570,12 +586,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
         const int q = seg & 1;
         // the accumulator of segment seg - 2 must have been read out
         if (first && seg >= 2 &&
-            !mbar_wait_ab(smem_u32(&bars.accfree[q]), ((seg >> 1) - 1) & 1, ab)) {
+            !mbar_wait_ab(smem_u32(&bars.accfree[q]), ((seg >> 1) - 1) & 1, ab, budget)) {
           ok = false;
           break;
         }
         const int s = i % kS32;
-        if (!mbar_wait_ab(smem_u32(&bars.afull[s]), (i / kS32) & 1, ab)) {
+        if (!mbar_wait_ab(smem_u32(&bars.afull[s]), (i / kS32) & 1, ab, budget)) {
           ok = false;
           break;
         }
@@ -606,7 +622,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
     const int nsegs = nunits > 0 ? (int)((u1 - 1) / C) - t_first + 1 : 0;
     for (int sg = 0; sg < nsegs; ++sg) {
       const int q = sg & 1;
-      const bool ok = mbar_wait_ab(smem_u32(&bars.accf[q]), (sg >> 1) & 1, ab);
+      const bool ok = mbar_wait_ab(smem_u32(&bars.accf[q]), (sg >> 1) & 1, ab, budget);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int t = t_first + sg;
@@ -646,7 +662,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) contract_tma_kernel(
       const int s = i % kS32;
       // the copies of chunk i have landed; the producer waited for the MMAs of
       // chunk i - kS32 before issuing them, so A stage s is free as well
-      const bool ok = mbar_wait_ab(smem_u32(&bars.full[s]), (i / kS32) & 1, ab);
+      const bool ok = mbar_wait_ab(smem_u32(&bars.full[s]), (i / kS32) & 1, ab, budget);
       if (!__all_sync(0xffffffffu, ok)) break;
       const unsigned char* st = ring + s * kStageBytesP;
       float x[16];
@@ -785,7 +801,7 @@ bool tc_contract_tma_ok(int n) { return tma_ok(nullptr, n) && encode_fn() != nul
 int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
                    const unsigned long long* Vs, const unsigned char* Bop, const float* w,
                    const float* wpad, int bb, const TcPlan* p, int klen, int splits, float* Pp,
-                   cudaStream_t st) {
+                   long long budget, cudaStream_t st) {
   using namespace umma;
   set_attrs();
   int* status = status_word_ptr();
@@ -793,7 +809,8 @@ int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
   if (p) {
     if (!make_tmap(&tm, R, m, n, 0)) return EXTERND_ERR_CUDA;
     contract_tma_kernel<0><<<p->G, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, w ? wpad : nullptr, bb,
-                                                            p->C, p->U, p->S, Pp, status);
+                                                            p->C, p->U, p->S, Pp, status,
+                                                            budget > 0 ? budget : kWaitBudget);
   } else {
     contract_kernel<0><<<dim3((unsigned)((m + kM - 1) / kM), (unsigned)splits), umma::kThreads,
                          kSmemBytes, st>>>(R, m, n, Vm, Vs, w, bb, klen, Pp, status);
@@ -803,7 +820,7 @@ int tc_contract_rv(const float* R, int m, int n, const unsigned long long* Vm,
 
 int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
                     const unsigned long long* Us, const unsigned char* Bop, int bb, const TcPlan* p,
-                    int klen, int splits, float* Qp, cudaStream_t st) {
+                    int klen, int splits, float* Qp, long long budget, cudaStream_t st) {
   using namespace umma;
   set_attrs();
   int* status = status_word_ptr();
@@ -811,7 +828,8 @@ int tc_contract_rtu(const float* R, int m, int n, const unsigned long long* Um,
   if (p) {
     if (!make_tmap(&tm, R, m, n, 1)) return EXTERND_ERR_CUDA;
     contract_tma_kernel<1><<<p->G, kThreadsP, kSmemP, st>>>(tm, m, n, Bop, nullptr, bb, p->C, p->U,
-                                                            p->S, Qp, status);
+                                                            p->S, Qp, status,
+                                                            budget > 0 ? budget : kWaitBudget);
   } else {
     contract_kernel<1><<<dim3((unsigned)((n + kM - 1) / kM), (unsigned)splits), umma::kThreads,
                          kSmemBytes, st>>>(R, m, n, Um, Us, nullptr, bb, klen, Qp, status);

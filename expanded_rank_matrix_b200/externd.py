@@ -35,7 +35,7 @@ MAX_SWEEPS = 64
 EXPORTS = ("externd_rank", "externd_decompose", "externd_decompose_ex", "externd_decompose_traced",
            "externd_reconstruct", "externd_sync_status", "externd_decompose_noalloc",
            "externd_decompose_block_traced", "externd_rank_for_energy",
-           "externd_ternary_apply", "externd_probe_read_bandwidth")
+           "externd_ternary_apply", "externd_probe_read_bandwidth", "externd_release_cache")
 
 _lib = None
 _vp = ctypes.c_void_p
@@ -77,7 +77,7 @@ def load(path: str = LIB_PATH):
     L.externd_decompose_noalloc.restype = ctypes.c_int
     L.externd_decompose_block_traced.argtypes = [_vp, _i64, _i64, ctypes.c_float, ctypes.c_float,
                                                  ctypes.c_int, _vp, ctypes.c_int, ctypes.c_uint,
-                                                 _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
+                                                 _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _i64, _vp]
     L.externd_decompose_block_traced.restype = ctypes.c_int
     L.externd_rank_for_energy.argtypes = [_vp, _i64, ctypes.c_double, _vp, _vp]
     L.externd_rank_for_energy.restype = ctypes.c_int
@@ -88,6 +88,8 @@ def load(path: str = LIB_PATH):
     L.externd_probe_read_bandwidth.restype = ctypes.c_int
     L.externd_sync_status.argtypes = [_vp]
     L.externd_sync_status.restype = ctypes.c_int
+    L.externd_release_cache.argtypes = []
+    L.externd_release_cache.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -323,6 +325,13 @@ def sync_status(stream: Optional[torch.cuda.Stream] = None) -> int:
     return int(load().externd_sync_status(_stream(stream)))
 
 
+def release_cache() -> int:
+    """externd_release_cache: drops the block path's cached graphs (with
+    their workspaces) and trims the inference scratch pools; returns the C
+    status."""
+    return int(load().externd_release_cache())
+
+
 # --- decoding of packed outputs (host side, for inspection and tests) -------
 
 def unpack_planes(packed: np.ndarray, length: int) -> np.ndarray:
@@ -368,7 +377,7 @@ class BlockTrace:
 def decompose_block_traced(A: torch.Tensor, mu: float, tau: float, iters: int, block: int,
                            trace_blocks: Sequence[int], w: Optional[torch.Tensor] = None,
                            stream: Optional[torch.cuda.Stream] = None, check: bool = True,
-                           flags: int = 0):
+                           flags: int = 0, wait_budget: int = 0):
     m, n = A.shape
     k = rank(m, n, mu)
     out = alloc_factors(m, n, k, A.device)
@@ -383,13 +392,15 @@ def decompose_block_traced(A: torch.Tensor, mu: float, tau: float, iters: int, b
         _ptr(out.packed_C),
         _ptr(out.D), _ptr(out.energy), nt,
         blocks.ctypes.data_as(ctypes.c_void_p) if nt else None, _ptr(uv) if nt else None,
-        _ptr(rows) if nt else None, _stream(stream))
+        _ptr(rows) if nt else None, wait_budget, _stream(stream))
     if rc != OK:
         raise ExterndError(rc, "externd_decompose_block_traced")
     status = sync_status(stream)
     if check and status != OK:
         raise ExterndError(status, "externd_decompose_block_traced (device)")
-    return out, BlockTrace(blocks, uv[:nt], rows[:nt], iters, block)
+    tr = BlockTrace(blocks, uv[:nt], rows[:nt], iters, block)
+    tr.status = status
+    return out, tr
 
 
 def _mask_codes(mask: np.ndarray, sign: np.ndarray, bb: int) -> np.ndarray:

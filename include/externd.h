@@ -114,7 +114,8 @@ int64_t externd_rank(int64_t m, int64_t n, float mu);
  * device's graph memory pool.  The replay reads A and w at launch time, so
  * new contents under the same pointers are honoured.  Calls on a stream that
  * is being captured run directly (they become part of the caller's graph);
- * setting the environment variable EXTERND_NO_GRAPH=1 disables replay.
+ * setting the environment variable EXTERND_NO_GRAPH=1 disables replay, and
+ * externd_release_cache() drops the cached graphs with their memory.
  */
 int externd_decompose(const float* A, int64_t m, int64_t n, float mu, float tau, int iters,
                       const float* w, int block, uint32_t* packed_B, uint32_t* packed_C,
@@ -201,13 +202,20 @@ int externd_decompose_traced(const float* A, int64_t m, int64_t n, float mu, flo
  *                and the n mask and n sign words of V_t.
  *   trace_rows   [ntrace][block] int32 (device) out: the block's start rows in
  *                order (energy descending, index ascending).
+ *   wait_budget  upper bound, in SM clock cycles, on the tensor-core
+ *                contractions' waits for their pipeline stages; 0 selects the
+ *                default (about 1 s).  A wait that runs out sets
+ *                EXTERND_ERR_TIMEOUT; the CTA then drains its own copies and
+ *                MMAs (with the default bound), frees its tensor memory and
+ *                returns, so the call completes with undefined outputs.
  */
 int externd_decompose_block_traced(const float* A, int64_t m, int64_t n, float mu, float tau,
                                    int iters, const float* w, int block, unsigned flags,
                                    uint32_t* packed_B,
                                    uint32_t* packed_C, float* D, double* energy_trace,
                                    int64_t ntrace, const int64_t* trace_block, uint64_t* trace_uv,
-                                   int32_t* trace_rows, externd_stream_t stream);
+                                   int32_t* trace_rows, int64_t wait_budget,
+                                   externd_stream_t stream);
 
 /*
  * externd_reconstruct -- A_hat = B diag(D) C from the packed factors (the
@@ -266,10 +274,14 @@ int externd_ternary_apply(const uint32_t* packed_B, const uint32_t* packed_C, co
  * allocating routine.  The caller still owns and passes every input and
  * output, with the same meaning as for externd_decompose.
  *
- * Limits: the residual must fit in the persistent grid's shared memory
- * (about 26 MB of fp32 on a B200, e.g. 2560 x 2560) and the exchange ring
- * must fit in the fixed array; larger problems return
- * EXTERND_ERR_SCRATCH_LIMIT without launching anything.
+ * Limits: the launch plan is the cheapest one (of those externd_decompose
+ * chooses among) that keeps the whole residual in the persistent grid's
+ * shared memory (about 26 MB of fp32 on a B200, e.g. 2560 x 2560) and whose
+ * exchange ring fits in the fixed array; when no plan qualifies the call
+ * returns EXTERND_ERR_SCRATCH_LIMIT without launching anything.  Where
+ * externd_decompose's own plan qualifies (2560 x 2560 and smaller square
+ * problems do) both entry points run the same plan and give identical
+ * factors.
  * The first call on a device looks up the device address of the fixed array
  * (a one-time set-up per device, done with that device current); make that
  * first call before any stream capture.
@@ -322,6 +334,20 @@ int externd_rank_for_energy(const double* energy_trace, int64_t k, double target
 #define EXTERND_PROBE_L2 1
 int externd_probe_read_bandwidth(int kind, const void* buf, int64_t bytes, int reps,
                                  int64_t* bytes_read, externd_stream_t stream);
+
+/*
+ * externd_release_cache -- gives back the device memory the library keeps
+ * between calls: destroys every CUDA graph that block-mode replay has
+ * captured (each holds its own workspace, including a copy of the residual,
+ * in its device's graph memory pool), returns that graph memory to the
+ * devices (cudaDeviceGraphMemTrim), and trims the inference scratch pools
+ * to zero (cudaMemPoolTrimTo).  Work already queued keeps what it uses:
+ * destruction and trimming leave alone memory that queued work still needs.
+ * Later calls capture and allocate again as usual.  Not stream-ordered;
+ * safe to call from any thread.  Returns EXTERND_OK, or EXTERND_ERR_CUDA if a trim failed (the caches are
+ * emptied regardless).
+ */
+int externd_release_cache(void);
 
 /*
  * externd_sync_status -- synchronises `stream`, then returns and clears the

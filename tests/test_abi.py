@@ -92,7 +92,7 @@ def test_variant_and_sweep_argument_checks(lib):
     assert L.externd_decompose_ex(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 0, 2, fake, fake, fake, fake,
                                   nul, nul) == X.ERR_INVALID_ARG
     assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, 8, fake, fake,
-                                            fake, fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+                                            fake, fake, 0, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
 
 
 def test_block_argument_checks(lib):
@@ -106,13 +106,13 @@ def test_block_argument_checks(lib):
                                nul) == X.ERR_INVALID_ARG
     # the block-traced entry is block-mode only and needs its trace buffers
     assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 1, 0, fake, fake, fake,
-                                            fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+                                            fake, 0, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
     assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, 0, fake, fake,
-                                            fake, fake, 2, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+                                            fake, fake, 2, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
     assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 16, 0, fake, fake,
-                                            fake, fake, -1, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+                                            fake, fake, -1, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
     assert L.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, nul, 65, 0, fake, fake,
-                                            fake, fake, 0, nul, nul, nul, nul) == X.ERR_INVALID_ARG
+                                            fake, fake, 0, nul, nul, nul, 0, nul) == X.ERR_INVALID_ARG
 
 
 def test_unpack_planes_layout():
@@ -166,3 +166,15 @@ def test_probe_argument_checks(lib):
     mis = ctypes.c_void_p((1 << 20) + 8)
     assert L.externd_probe_read_bandwidth(X.PROBE_L2, mis, 1 << 20, 1, ctypes.byref(out),
                                           None) == X.ERR_INVALID_ARG
+
+
+def test_block_wait_budget_must_not_be_negative(lib):
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.externd_decompose_block_traced(fake, 64, 64, 1.0, 0.5, 2, None, 16, 0, fake, fake,
+                                              fake, fake, 0, None, None, None, -1,
+                                              None) == X.ERR_INVALID_ARG
+
+
+def test_release_cache_with_nothing_cached(lib):
+    # no graph captured and no pool created in this process: nothing to do
+    assert lib.externd_release_cache() == X.OK

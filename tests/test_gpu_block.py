@@ -173,3 +173,51 @@ def test_graph_replay_matches_direct(monkeypatch):
             assert torch.equal(a, b)
     for a, b in zip(scaled, direct_scaled):
         assert torch.equal(a, b)
+
+
+def test_contraction_wait_budget_runs_out_cleanly():
+    """A one-cycle budget on the tensor-core contractions' pipeline waits: the
+    first stage a converter waits for has not landed yet, so the call ends
+    with EXTERND_ERR_TIMEOUT; the CTAs drain their own copies and MMAs and free
+    their tensor memory, and the next call on the same context is exact."""
+    A = _dev(W.llm_like(640, 512, 21, n_outliers=2))
+    f, tr = X.decompose_block_traced(A, 0.25, 0.5, 2, 32, [], check=False, wait_budget=1)
+    assert tr.status == X.ERR_TIMEOUT
+    g = X.decompose(A, 0.25, 0.5, 2, block=32)
+    assert X.sync_status() == X.OK
+    ref = X.decompose(A, 0.25, 0.5, 2, block=32)
+    assert torch.equal(g.D, ref.D) and float(g.energy[-1]) > 0.3
+
+
+def test_direct_contraction_many_ctas(oracle):
+    """Rows of R not 16-byte aligned (n % 4 != 0) take the direct contraction,
+    which keeps several CTAs on an SM: 2000 x 1998 launches far more CTAs than
+    SMs.  The first two 64-wide blocks are teacher-forced."""
+    A = W.llm_like(2000, 1998, 33, n_outliers=3)
+    rep, f = block_teacher_forced(oracle, A, 0.5, 0.5, 2, 64, blocks=[0, 1])
+    print(f"2000x1998 b=64 (direct path): band {rep.band_total} mismatch {rep.band_mismatch} "
+          f"max D rel {rep.d_rel_max:.2e}")
+    assert rep.ok, rep.bad
+
+
+def test_release_cache_drops_graphs():
+    """externd_release_cache destroys the captured graphs and trims their
+    memory; calls after it run directly, capture again and replay, with the
+    same results as before."""
+    A = _dev(W.llm_like(640, 512, 22, n_outliers=2))
+    k = X.rank(640, 512, 0.5)
+    f = X.alloc_factors(640, 512, k, A.device)
+    for _ in range(3):  # direct, capture + replay, replay
+        X.decompose_into(f, A, 0.5, 0.5, 3, block=32)
+    before = [t.clone() for t in (f.packed_B, f.packed_C, f.D, f.energy)]
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    assert X.release_cache() == X.OK
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] >= free0
+    assert X.release_cache() == X.OK  # nothing left to release
+    for _ in range(3):
+        X.decompose_into(f, A, 0.5, 0.5, 3, block=32)
+        for a, b in zip(before, (f.packed_B, f.packed_C, f.D, f.energy)):
+            assert torch.equal(a, b)
+    assert X.sync_status() == X.OK

@@ -155,11 +155,12 @@ def test_nonfinite_input_reports_status():
 
 
 def test_wait_budget_runs_out_cleanly():
-    # a one-cycle budget makes the cross-CTA waits give up: the call must end
-    # with EXTERND_ERR_TIMEOUT and leave the context usable
+    # a one-cycle budget makes the cross-CTA waits give up: the first wait of
+    # every CTA is on data another SM writes later, so the call must end with
+    # EXTERND_ERR_TIMEOUT -- and leave the context usable
     A = _dev(W.llm_like(512, 512, 9))
     f, tr, status = X.decompose_traced(A, 1.0, 0.5, 2, [], wait_budget=1, check=False)
-    assert status in (X.ERR_TIMEOUT, X.OK)
+    assert status == X.ERR_TIMEOUT
     f2 = X.decompose(A, 1.0, 0.5, 2)
     assert X.sync_status() == X.OK
     assert float(f2.energy[-1]) > 0.5
