@@ -56,8 +56,7 @@ __device__ double block_sum_d(double x, double* sh) {
 // ---- setup: R = A, row-energy partials per column chunk, validity -----------
 // Row energies are kept as partials over column chunks of kChunk columns,
 // rhop[chunk][row], summed in chunk order where a full energy is needed.
-constexpr int kChunk = 1024;  // deflate_kernel assumes 4 x 256 threads
-static_assert(kChunk == 4 * 256, "deflate fill layout");
+constexpr int kChunk = 256;
 __global__ void setup_kernel(const float* __restrict__ A, float* __restrict__ R, int m, int n,
                              const float* __restrict__ w, double* __restrict__ rhop,
                              int* __restrict__ bad) {
@@ -115,8 +114,10 @@ __global__ void __launch_bounds__(1024) select_rows_kernel(const double* __restr
   const int tid = threadIdx.x;
   double part = 0.0;
   for (int i0 = 0; i0 < m; i0 += 4096) {
-    // four rows per thread per round, every partial load in flight together
+    // four rows per thread per round; eight chunks' partial loads in flight
+    // together (the sums still run in chunk order)
     double r[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 8
     for (int c = 0; c < nch; ++c) {
       double v[4];
 #pragma unroll
@@ -388,54 +389,90 @@ __global__ void gram_kernel(const uint32_t* __restrict__ planes, int W, int bb,
 // ---- in-place Gauss-Jordan inverse of an SPD matrix (no pivoting) ----------
 // The bb x bb matrix (bb <= 64, zero padded to 64 x 64) lives in registers of
 // a 256-thread CTA: warp w holds rows 8w .. 8w+7, lane holds columns lane and
-// lane + 32.  Pivot k: its owner warp publishes row k to shared memory (two
-// alternating buffers, so one barrier per pivot suffices); every thread then
-// forms the scaled pivot row n = a_k / a_kk (n_k = 1 / a_kk) for its columns
-// and updates its rows, a_ij <- a_ij - a_ik n_j for j != k and
-// a_ik <- -a_ik n_k.  After bb pivots the registers hold the inverse.
-__device__ __forceinline__ void gj_inverse(double (&a)[8][2], int bb, double* prow) {
+// lane + 32.  The pivots are taken in blocks of eight, K = 8w .. 8w+7, which
+// are exactly warp w's rows.  Block K: warp w runs the eight in-place pivot
+// steps on its own rows alone (for pivot k: n = a_k / a_kk with n_k = 1 / a_kk,
+// row k <- n, and a_ij <- a_ij - a_ik n_j (j != k), a_ik <- -a_ik n_k on the
+// block's other rows; the factors come by warp shuffles).  Those rows then
+// hold [A_KK^-1, A_KK^-1 A_KJ] and are published to shared memory, together
+// with every other row's factors a_iK (before the block).  Each other row
+// takes the block's eight steps at once, a_ij <- [j not in K] a_ij -
+// sum_k a_ik P_kj, which is the same elimination regrouped (the Schur
+// complement update).  Two barriers per block; after all blocks the
+// registers hold the inverse.  `sm` holds 1024 doubles.
+__device__ __forceinline__ void gj_inverse(double (&a)[8][2], int bb, double* sm) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  // row 0 is published up front; row k + 1 by its owner right after it has
-  // been updated in step k (selecting a register row by a runtime index
-  // would force the matrix into local memory)
-  if (wid == 0) {
-    prow[lane] = a[0][0];
-    prow[lane + 32] = a[0][1];
-  }
-  for (int k = 0; k < bb; ++k) {
-    __syncthreads();
-    const double* pr = prow + (k & 1) * kMaxB;
-    const double p = 1.0 / pr[k];
-    const double n0 = lane == k ? p : pr[lane] * p;
-    const double n1 = lane + 32 == k ? p : pr[lane + 32] * p;
-    const int lk = k & 31;
-    const bool hi = k >= 32;
-    double* nx = prow + ((k + 1) & 1) * kMaxB;
+  double* const P = sm;             // [8][64]: the block's transformed rows
+  double* const F = sm + 8 * kMaxB;  // [64 rows][8]: each row's factors a_iK
+  const int nblk = (bb + 7) >> 3;
+  for (int K = 0; K < nblk; ++K) {
+    const int kb = 8 * K, nk = min(8, bb - kb);
+    const int lk = kb & 31;  // lane holding column kb (columns kb .. kb+7: lanes lk .. lk+7)
+    const bool hk = kb >= 32;
+    if (wid == K) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const double f0 = __shfl_sync(0xffffffffu, a[q][0], lk);
-      const double f1 = __shfl_sync(0xffffffffu, a[q][1], lk);
-      const double f = hi ? f1 : f0;
-      if (wid * 8 + q == k) {
-        a[q][0] = n0;
-        a[q][1] = n1;
-      } else {
-        a[q][0] = (lane == k ? 0.0 : a[q][0]) - f * n0;
-        a[q][1] = (lane + 32 == k ? 0.0 : a[q][1]) - f * n1;
+      for (int kk = 0; kk < 8; ++kk) {
+        if (kk < nk) {
+          const int k = kb + kk;
+          const double piv = __shfl_sync(0xffffffffu, hk ? a[kk][1] : a[kk][0], lk + kk);
+          const double p = 1.0 / piv;
+          const double n0 = lane == k ? p : a[kk][0] * p;
+          const double n1 = lane + 32 == k ? p : a[kk][1] * p;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const double f = __shfl_sync(0xffffffffu, hk ? a[q][1] : a[q][0], lk + kk);
+            if (q == kk) {
+              a[q][0] = n0;
+              a[q][1] = n1;
+            } else {
+              a[q][0] = (lane == k ? 0.0 : a[q][0]) - f * n0;
+              a[q][1] = (lane + 32 == k ? 0.0 : a[q][1]) - f * n1;
+            }
+          }
+        }
       }
-      if (wid * 8 + q == k + 1) {
-        nx[lane] = a[q][0];
-        nx[lane + 32] = a[q][1];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        P[q * kMaxB + lane] = a[q][0];
+        P[q * kMaxB + lane + 32] = a[q][1];
+      }
+    } else if (lane >= lk && lane < lk + 8) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) F[(wid * 8 + q) * 8 + (lane - lk)] = hk ? a[q][1] : a[q][0];
+    }
+    __syncthreads();
+    if (wid != K) {
+      double pv[8][2];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        pv[kk][0] = P[kk * kMaxB + lane];
+        pv[kk][1] = P[kk * kMaxB + lane + 32];
+      }
+      const bool in0 = lane >= kb && lane < kb + 8, in1 = lane + 32 >= kb && lane + 32 < kb + 8;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const double2* fr = (const double2*)(F + (wid * 8 + q) * 8);
+        const double2 f01 = fr[0], f23 = fr[1], f45 = fr[2], f67 = fr[3];
+        const double f[8] = {f01.x, f01.y, f23.x, f23.y, f45.x, f45.y, f67.x, f67.y};
+        double x0 = in0 ? 0.0 : a[q][0], x1 = in1 ? 0.0 : a[q][1];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          x0 -= f[kk] * pv[kk][0];
+          x1 -= f[kk] * pv[kk][1];
+        }
+        a[q][0] = x0;
+        a[q][1] = x1;
       }
     }
+    __syncthreads();  // P and F are rewritten by the next block
   }
-  __syncthreads();
+  __syncthreads();  // (also when bb == 0)
 }
 
 // S = (G + eps I)^-1 with eps = 1e-6 tr(G) / bb (1 when the trace is 0).
 __global__ void __launch_bounds__(256, 1) inv_kernel(const double* __restrict__ G, int bb,
                                                   double* __restrict__ S) {
-  __shared__ double prow[2 * kMaxB];
+  __shared__ __align__(16) double prow[16 * kMaxB];
   __shared__ double eps;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (wid == 0) {
@@ -469,76 +506,88 @@ __global__ void __launch_bounds__(256, 1) inv_kernel(const double* __restrict__ 
 }
 
 // ---- targets: T[x][l] = sum_l2 (sum_s Xp[s][x][l2]) S[l2][l] (fp64) ----------
-// 64 rows per CTA, two CTAs per SM (one wave for up to 2 x SMs x 64 rows).
-// The split-K partials are summed (split order, fp64) into a transposed tile
-// Xt[l2][row] in shared memory next to S -- each thread loads 4 consecutive
-// columns of 4 rows, float4 per split, all splits in flight (NS >= splits is
-// a compile-time bound).  Thread (rg, cg) then forms the 4 x 4 block rows
-// 4rg.., columns 4cg.. of T: 16 independent fp64 chains per thread.  Each CTA
-// writes its column sums of squares; the last CTA to finish (ticket counter)
-// sums those partials in CTA order and writes the column thresholds
+// The rows are split evenly over at most one CTA per SM: CTA c takes rows
+// [c rpc, (c+1) rpc) with rpc <= 80, so no SM holds twice the work of
+// another.  The split-K / stream-K partials are summed (in partial order,
+// fp64) into a transposed tile Xt[l2][row] in shared memory next to S -- each
+// thread loads 4 consecutive columns of 4 rows, float4 per partial, all
+// partials in flight (NS >= partials is a compile-time bound).  Thread
+// (rg, cg) then forms the 4 x 4 block rows 4rg.., columns 4cg.. of T: 16
+// independent fp64 chains per thread.  Each CTA writes its column sums of
+// squares (stat 0) or of absolute values (stat 1); the last CTA to finish
+// (ticket counter) adds those partials in a fixed order -- thread (q, l)
+// takes CTAs q, q + 5, q + 10, ... in CTA order with all its loads in
+// flight, then the five sums in q order -- and writes the column thresholds
 // thr[l] = tau * rms(T[:, l]) (stat 0) or tau * mean |T[:, l]| (stat 1), then
-// rearms the counter.  With Xout set, the split-summed X (rows x bb, fp64) is
-// stored as well.  With wsc set, row x of T is scaled by wsc[x] before it is
-// stored and measured (the naive weighted V-step thresholds W times the
+// rearms the counter.  With Xout set, the partial-summed X (rows x bb, fp64)
+// is stored as well.  With wsc set, row x of T is scaled by wsc[x] before it
+// is stored and measured (the naive weighted V-step thresholds W times the
 // target).
-constexpr int kTgtRows2 = 64;  // rows per CTA of target_kernel
+constexpr int kTgtThreads = 320;     // 20 row groups x 16 column groups
+constexpr int kTgtMaxRows = 80;      // rows per CTA at most (20 groups x 4)
+constexpr int kTgtRedGroups = kTgtThreads / kMaxB;  // 5 summing groups in the last CTA
+constexpr int kTgtRedLoads = 32;     // loads in flight per thread in the last CTA
 constexpr int kMaxSplits = kMaxSegs;  // partials per output row (split-K or stream-K)
-constexpr int kXs = kTgtRows2 + 2;  // padded row of the transposed tile (16-byte aligned)
+constexpr int kXs = kTgtMaxRows + 2;  // padded row of the transposed tile (16-byte aligned)
+// rows per CTA for `rows` rows on nsm SMs
+inline int target_rpc(int rows, int nsm) {
+  const int r = (rows + nsm - 1) / std::max(nsm, 1);
+  return std::max(1, std::min(kTgtMaxRows, r));
+}
 // Partials: split-K layout Xp[split][row][bb] (sk == 0, `splits` of them) or
 // stream-K layout Xp[(t Sslots + slot) 128 + row % 128][bb] with the tile's
 // segment count from the plan (C, U, G) (sk != 0).
 template <int NS>
-__global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict__ Xp, int splits,
-                                                        int rows, int bb,
-                                                        const double* __restrict__ S, double tau,
-                                                        double* __restrict__ T,
-                                                        double* __restrict__ colss,
-                                                        unsigned* __restrict__ ticket,
-                                                        double* __restrict__ thr,
-                                                        double* __restrict__ Xout, int sk, int C,
-                                                        long long U, int G, int Sslots, int stat,
-                                                        const float* __restrict__ wsc) {
+__global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
+    const float* __restrict__ Xp, int splits, int rows, int rpc, int bb,
+    const double* __restrict__ S, double tau, double* __restrict__ T,
+    double* __restrict__ colss, unsigned* __restrict__ ticket, double* __restrict__ thr,
+    double* __restrict__ Xout, int sk, int C, long long U, int G, int Sslots, int stat,
+    const float* __restrict__ wsc) {
   extern __shared__ __align__(16) double tsh[];
-  double* Ss = tsh;                                                 // [64][64]: S[l2][l]
-  double* Xt = tsh + kMaxB * kMaxB;                                 // [64][kXs]
-  double (*part)[kMaxB] = (double (*)[kMaxB])(Xt + kMaxB * kXs);    // [16][64]
+  double* Ss = tsh;                                                    // [64][64]: S[l2][l]
+  double* Xt = tsh + kMaxB * kMaxB;                                    // [64][kXs]
+  double (*part)[kMaxB] = (double (*)[kMaxB])(Xt + kMaxB * kXs);       // [20][64]
   __shared__ bool last;
   const int tid = threadIdx.x;
-  const int x0 = blockIdx.x * kTgtRows2;
+  const int x0 = blockIdx.x * rpc, nr = min(rpc, rows - x0);
   {
-    double sv[16];
+    constexpr int kSL = (kMaxB * kMaxB + kTgtThreads - 1) / kTgtThreads;
+    double sv[kSL];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const int p = tid + 256 * q, l2 = p >> 6, lc = p & 63;
-      sv[q] = (l2 < bb && lc < bb) ? __ldg(S + l2 * bb + lc) : 0.0;
+    for (int q = 0; q < kSL; ++q) {
+      const int p = tid + kTgtThreads * q, l2 = p >> 6, lc = p & 63;
+      sv[q] = (p < kMaxB * kMaxB && l2 < bb && lc < bb) ? __ldg(S + l2 * bb + lc) : 0.0;
     }
 #pragma unroll
-    for (int q = 0; q < 16; ++q) Ss[tid + 256 * q] = sv[q];
+    for (int q = 0; q < kSL; ++q) {
+      const int p = tid + kTgtThreads * q;
+      if (p < kMaxB * kMaxB) Ss[p] = sv[q];
+    }
   }
   {
-    // thread: columns lq .. lq+3 (lq = 4 (tid % 16)), rows tid / 16 + 16 h
+    // thread: columns lq .. lq+3 (lq = 4 (tid % 16)), rows tid / 16 + 20 h
     const int lq = (tid & 15) * 4, rr = tid >> 4;
-    // 64-row CTAs never straddle a 128-row tile
-    const int nparts = sk ? umma::sk_nseg(x0 / umma::kM, C, U, G) : splits;
     const size_t sstride = sk ? (size_t)umma::kM * bb : (size_t)rows * bb;
     const bool vec = (bb & 3) == 0;
     constexpr int RPR = NS > 8 ? 1 : 2;  // rows per round: at most 64 floats in flight
 #pragma unroll 1
     for (int h0 = 0; h0 < 4; h0 += RPR) {
       float4 v[RPR][NS];
+      int np[RPR];
 #pragma unroll
       for (int h = 0; h < RPR; ++h) {
-        const int x = x0 + rr + 16 * (h0 + h);
-        const bool ok = x < rows && lq < bb;
+        const int r = rr + 20 * (h0 + h), x = x0 + r;
+        const bool ok = r < nr && lq < bb;
         const int xs = ok ? x : 0;
+        np[h] = sk ? umma::sk_nseg(xs / umma::kM, C, U, G) : splits;
         const size_t prow = sk ? ((size_t)(xs / umma::kM) * Sslots * umma::kM + xs % umma::kM)
                                : (size_t)xs;
         const float* src = Xp + prow * bb + (ok ? lq : 0);
 #pragma unroll
         for (int sp = 0; sp < NS; ++sp) {
           float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (ok && sp < nparts) {
+          if (ok && sp < np[h]) {
             const float* q = src + sp * sstride;
             if (vec) {
               t = __ldg((const float4*)q);
@@ -557,19 +606,19 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
         double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
 #pragma unroll
         for (int sp = 0; sp < NS; ++sp)
-          if (sp < nparts) {
+          if (sp < np[h]) {
             s0 += (double)v[h][sp].x;
             s1 += (double)v[h][sp].y;
             s2 += (double)v[h][sp].z;
             s3 += (double)v[h][sp].w;
           }
-        const int r = rr + 16 * (h0 + h);
+        const int r = rr + 20 * (h0 + h);
         Xt[(lq + 0) * kXs + r] = s0;
         Xt[(lq + 1) * kXs + r] = s1;
         Xt[(lq + 2) * kXs + r] = s2;
         Xt[(lq + 3) * kXs + r] = s3;
         const int x = x0 + r;
-        if (Xout && x < rows) {
+        if (Xout && r < nr) {
           const double sx[4] = {s0, s1, s2, s3};
 #pragma unroll
           for (int j = 0; j < 4; ++j)
@@ -585,28 +634,30 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+  if (4 * rg < nr) {
 #pragma unroll 2
-  for (int l2 = 0; l2 < bb; ++l2) {
-    const double2 xa = *(const double2*)(Xt + l2 * kXs + 4 * rg);
-    const double2 xb = *(const double2*)(Xt + l2 * kXs + 4 * rg + 2);
-    const double2 sa = *(const double2*)(Ss + l2 * kMaxB + 4 * cg);
-    const double2 sb = *(const double2*)(Ss + l2 * kMaxB + 4 * cg + 2);
-    const double xv[4] = {xa.x, xa.y, xb.x, xb.y}, svv[4] = {sa.x, sa.y, sb.x, sb.y};
+    for (int l2 = 0; l2 < bb; ++l2) {
+      const double2 xa = *(const double2*)(Xt + l2 * kXs + 4 * rg);
+      const double2 xb = *(const double2*)(Xt + l2 * kXs + 4 * rg + 2);
+      const double2 sa = *(const double2*)(Ss + l2 * kMaxB + 4 * cg);
+      const double2 sb = *(const double2*)(Ss + l2 * kMaxB + 4 * cg + 2);
+      const double xv[4] = {xa.x, xa.y, xb.x, xb.y}, svv[4] = {sa.x, sa.y, sb.x, sb.y};
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += xv[i] * svv[j];
+        for (int j = 0; j < 4; ++j) acc[i][j] += xv[i] * svv[j];
+    }
   }
   double cs[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int x = x0 + 4 * rg + i;
-    if (x < rows && wsc) {
-      const double ws = (double)wsc[x];
+    const int r = 4 * rg + i, x = x0 + r;
+    if (r < nr) {
+      if (wsc) {
+        const double ws = (double)wsc[x];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] *= ws;
-    }
-    if (x < rows) {
+        for (int j = 0; j < 4; ++j) acc[i][j] *= ws;
+      }
       if (bb == kMaxB) {
         *(double2*)(T + (size_t)x * bb + 4 * cg) = make_double2(acc[i][0], acc[i][1]);
         *(double2*)(T + (size_t)x * bb + 4 * cg + 2) = make_double2(acc[i][2], acc[i][3]);
@@ -624,7 +675,7 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
   __syncthreads();
   if (tid < kMaxB) {
     double c = 0.0;
-    for (int g = 0; g < 16; ++g) c += part[g][tid];
+    for (int g = 0; g < kTgtThreads / 16; ++g) c += part[g][tid];
     if (tid < bb) colss[(size_t)blockIdx.x * bb + tid] = c;
   }
   __syncthreads();
@@ -636,35 +687,38 @@ __global__ void __launch_bounds__(256, 2) target_kernel(const float* __restrict_
   if (!last) return;
   __threadfence();
   {
-    // thread (q, l) sums the partials of CTAs b = q mod 4 in CTA order, eight
-    // loads in flight; the four sums are then added in q order
-    const int l = tid & 63, q = tid >> 6;
+    const int l = tid & 63, q = tid / kMaxB;
+    const int nb = (int)gridDim.x;
     double c = 0.0;
     if (l < bb) {
-      const unsigned nb = gridDim.x;
-      unsigned b = q;
-      for (; b + 28 < nb; b += 32) {
-        double v[8];
+      for (int b0 = q; b0 < nb; b0 += kTgtRedGroups * kTgtRedLoads) {
+        double v[kTgtRedLoads];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldcg(colss + (size_t)(b + 4 * u) * bb + l);
+        for (int u = 0; u < kTgtRedLoads; ++u) {
+          const int b = b0 + kTgtRedGroups * u;
+          v[u] = b < nb ? __ldcg(colss + (size_t)b * bb + l) : 0.0;
+        }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) c += v[u];
+        for (int u = 0; u < kTgtRedLoads; ++u)
+          if (b0 + kTgtRedGroups * u < nb) c += v[u];
       }
-      for (; b < nb; b += 4) c += __ldcg(colss + (size_t)b * bb + l);
     }
     part[q][l] = c;
     __syncthreads();
     if (tid < bb) {
-      const double t4 = ((part[0][tid] + part[1][tid]) + part[2][tid]) + part[3][tid];
-      thr[tid] = stat ? tau * (t4 / (double)rows) : tau * sqrt(t4 / (double)rows);
+      double t5 = part[0][tid];
+#pragma unroll
+      for (int g = 1; g < kTgtRedGroups; ++g) t5 += part[g][tid];
+      thr[tid] = stat ? tau * (t5 / (double)rows) : tau * sqrt(t5 / (double)rows);
     }
   }
   if (tid == 0) *ticket = 0u;
 }
-constexpr size_t kTgtSmem = sizeof(double) * (kMaxB * kMaxB + kMaxB * kXs + 16 * kMaxB);
-// the target kernel instantiated for a split-count bound
-typedef void (*TargetFn)(const float*, int, int, int, const double*, double, double*, double*,
-                         unsigned*, double*, double*, int, int, long long, int, int, int,
+constexpr size_t kTgtSmem =
+    sizeof(double) * (kMaxB * kMaxB + kMaxB * kXs + (kTgtThreads / 16) * kMaxB);
+// the target kernel instantiated for a partial-count bound
+typedef void (*TargetFn)(const float*, int, int, int, int, const double*, double, double*,
+                         double*, unsigned*, double*, double*, int, int, long long, int, int, int,
                          const float*);
 inline TargetFn target_for(int splits) {
   if (splits <= 1) return target_kernel<1>;
@@ -675,60 +729,77 @@ inline TargetFn target_for(int splits) {
 }
 
 // ---- ternary codes: 64-bit masks per entry and packed planes -----------------
-// One warp per 32 entries (one plane word): lanes read the entry's T row
-// (coalesced) and ballot the threshold tests, so lane r ends up holding the
-// masks of entry r; 64 more ballots per warp transpose them into planes.
-__global__ void tern_kernel(const double* __restrict__ T, int rows, int bb,
-                            const double* __restrict__ thr, u64* __restrict__ Mk,
-                            u64* __restrict__ Sg, uint32_t* __restrict__ planes, int W,
-                            unsigned char* __restrict__ bop) {
-  const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= W) return;
+// One CTA of 8 warps per 32 entries (one plane word t).  Warp w thresholds
+// entries 4w .. 4w+3: lane l reads T[x][l] and T[x][l + 32] (coalesced), and
+// four ballots give entry x's mask and sign words directly.  The 32 entries'
+// words meet in shared memory; warp w then transposes components
+// 8w .. 8w+7 into plane words (one ballot per component and plane), and every
+// thread writes one 16-byte group of the word's bf16 B chunk.
+__global__ void __launch_bounds__(256) tern_kernel(const double* __restrict__ T, int rows, int bb,
+                                                   const double* __restrict__ thr,
+                                                   u64* __restrict__ Mk, u64* __restrict__ Sg,
+                                                   uint32_t* __restrict__ planes, int W,
+                                                   unsigned char* __restrict__ bop) {
+  __shared__ u64 mk_s[32], sg_s[32];
+  __shared__ uint32_t om_s[kMaxB], os_s[kMaxB];
+  const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  double v0[4], v1[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int x = t * 32 + 4 * wid + q;
+    v0[q] = (x < rows && lane < bb) ? T[(size_t)x * bb + lane] : 0.0;
+    v1[q] = (x < rows && lane + 32 < bb) ? T[(size_t)x * bb + lane + 32] : 0.0;
+  }
   const double th0 = lane < bb ? thr[lane] : 0.0, th1 = lane + 32 < bb ? thr[lane + 32] : 0.0;
-  u64 mk = 0ull, sg = 0ull;
-#pragma unroll 8
-  for (int r = 0; r < 32; ++r) {
-    const int x = t * 32 + r;
-    double v0 = 0.0, v1 = 0.0;
-    if (x < rows) {
-      if (lane < bb) v0 = T[(size_t)x * bb + lane];
-      if (lane + 32 < bb) v1 = T[(size_t)x * bb + lane + 32];
-    }
-    const bool a0 = lane < bb && fabs(v0) > th0, a1 = lane + 32 < bb && fabs(v1) > th1;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const bool a0 = lane < bb && fabs(v0[q]) > th0, a1 = lane + 32 < bb && fabs(v1[q]) > th1;
     const uint32_t m0 = __ballot_sync(0xffffffffu, a0), m1 = __ballot_sync(0xffffffffu, a1);
-    const uint32_t s0 = __ballot_sync(0xffffffffu, a0 && v0 < 0.0);
-    const uint32_t s1 = __ballot_sync(0xffffffffu, a1 && v1 < 0.0);
-    if (lane == r) {
-      mk = (u64)m0 | ((u64)m1 << 32);
-      sg = (u64)s0 | ((u64)s1 << 32);
+    const uint32_t s0 = __ballot_sync(0xffffffffu, a0 && v0[q] < 0.0);
+    const uint32_t s1 = __ballot_sync(0xffffffffu, a1 && v1[q] < 0.0);
+    if (lane == 0) {
+      mk_s[4 * wid + q] = (u64)m0 | ((u64)m1 << 32);
+      sg_s[4 * wid + q] = (u64)s0 | ((u64)s1 << 32);
     }
   }
-  const int x = t * 32 + lane;
-  if (x < rows) {
-    Mk[x] = mk;
-    Sg[x] = sg;
+  __syncthreads();
+  const u64 mk = mk_s[lane], sg = sg_s[lane];  // entry t * 32 + lane (0 past the end)
+  if (wid == 0 && t * 32 + lane < rows) {
+    Mk[t * 32 + lane] = mk;
+    Sg[t * 32 + lane] = sg;
   }
-  uint32_t om[2] = {0u, 0u}, os[2] = {0u, 0u};
-  for (int l = 0; l < bb; ++l) {
+  uint32_t pm = 0u, ps = 0u;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const int l = 8 * wid + c;
     const uint32_t bm = __ballot_sync(0xffffffffu, (mk >> l) & 1ull);
     const uint32_t bs = __ballot_sync(0xffffffffu, (sg >> l) & 1ull);
-    if (lane == (l & 31)) {
-      om[l >> 5] = bm;
-      os[l >> 5] = bs;
+    if (lane == c) {
+      pm = bm;
+      ps = bs;
     }
   }
-  for (int h = 0; h < 2; ++h) {
-    const int l = lane + 32 * h;
+  if (lane < 8) {
+    const int l = 8 * wid + lane;
+    om_s[l] = pm;
+    os_s[l] = ps;
     if (l < bb) {
-      planes[(size_t)l * 2 * W + t] = om[h];
-      planes[(size_t)l * 2 * W + W + t] = os[h];
+      planes[(size_t)l * 2 * W + t] = pm;
+      planes[(size_t)l * 2 * W + W + t] = ps;
     }
   }
-  if (bop) write_bchunk(bop, t, lane, om, os);
+  if (!bop) return;
+  __syncthreads();
+  {
+    // thread -> component l = tid / 4, 8-entry group kg = tid % 4
+    const int l = tid >> 2, kg = tid & 3;
+    *(uint4*)(bop + (size_t)t * umma::kBBytes + umma::kmaj_off(l, kg * 8)) =
+        umma::bf16_codes8((om_s[l] >> (8 * kg)) & 0xffu, (os_s[l] >> (8 * kg)) & 0xffu);
+  }
 }
 
 // ---- r_l = u_l^T R W v_l = sum_j Q[j][l] w_j s_jl, per-CTA partials (64 rows)
+constexpr int kRpartRows = 64;
 // Q = R^T U, split-summed in fp64 by the last V-step target pass.
 __global__ void __launch_bounds__(256) rpart_kernel(const double* __restrict__ Q, int n, int bb,
                                                     const u64* __restrict__ Vm,
@@ -737,11 +808,11 @@ __global__ void __launch_bounds__(256) rpart_kernel(const double* __restrict__ Q
                                                     double* __restrict__ rp) {
   __shared__ double part[4][kMaxB];
   const int l = threadIdx.x & 63, rr = threadIdx.x >> 6;
-  const int x0 = blockIdx.x * kTgtRows2;
+  const int x0 = blockIdx.x * kRpartRows;
   double acc = 0.0;
   if (l < bb) {
 #pragma unroll 4
-    for (int t = 0; t < kTgtRows2 / 4; ++t) {
+    for (int t = 0; t < kRpartRows / 4; ++t) {
       const int j = x0 + rr + 4 * t;
       if (j < n) {
         const u64 mm = Vm[j];
@@ -769,7 +840,8 @@ __global__ void __launch_bounds__(256, 1) dsolve_kernel(const double* __restrict
                                                      double* __restrict__ energy,
                                                      float* __restrict__ dblk) {
   __shared__ double G[kMaxB * kMaxB];
-  __shared__ double r[kMaxB], ra[kMaxB], fcol[kMaxB], prow[2 * kMaxB];
+  __shared__ double r[kMaxB], ra[kMaxB], fcol[kMaxB];
+  __shared__ __align__(16) double prow[16 * kMaxB];
   __shared__ float dl[kMaxB];
   __shared__ int act[kMaxB];
   __shared__ int na;
@@ -845,116 +917,126 @@ __global__ void __launch_bounds__(256, 1) dsolve_kernel(const double* __restrict
 }
 
 // ---- ordered block deflation + next block's row-energy partials ------------
-// CTA = 8 warps x 2 rows each, over one chunk of kChunk columns whose V masks
-// sit in shared memory.  Row i's active components (u_il != 0) form a list
-// in ascending l with signed scales du_l = u_il d_l.  Each lane holds 4
-// entries x_j and, per entry, which active components meet v_jl = +1 (mask P)
-// or v_jl = -1 (mask N), split into 32-bit halves; the list is walked once
-// per half, so one component costs a bit test and a predicated fp32 add or
-// subtract per entry: x_j <- x_j - du_l (P) or x_j + du_l (N), in ascending l.
-__global__ void __launch_bounds__(256) deflate_kernel(float* __restrict__ R, int m, int n,
-                                                      const u64* __restrict__ Um,
-                                                      const u64* __restrict__ Us,
-                                                      const u64* __restrict__ Vm,
-                                                      const u64* __restrict__ Vs,
-                                                      const float* __restrict__ dblk,
-                                                      const float* __restrict__ w,
-                                                      double* __restrict__ rhop) {
-  __shared__ u64 vm[kChunk], vs[kChunk];
-  __shared__ float d[kMaxB];
-  __shared__ int ls_s[8][kMaxB];
-  __shared__ float du_s[8][kMaxB];
-  const int ch = blockIdx.y, j0 = ch * kChunk, j1 = min(n, j0 + kChunk), nj = j1 - j0;
+// CTA = 8 warps over 64 rows and one chunk of kChunk columns, walked in
+// sub-tiles of 128 columns.  Shared memory holds, per component l of the
+// block, the negated signed scales of the CTA's rows, nd_il = -(u_il d_l)
+// (0 where u_il = 0; stored twice, as a pair), and the sub-tile's V codes
+// expanded to fp32, vf_lj = v_jl in {-1, 0, +1}.  Warp w owns rows
+// 8w .. 8w+7 and lane t the columns 4t .. 4t+3 of the sub-tile, so a thread
+// holds an 8 x 4 block of R.  For l = 0, 1, ..., b-1 in order it takes
+// x <- fma(nd_il, vf_lj, x) on column pairs (__ffma2_rn).  The product is
+// exact (vf is -1, 0 or +1), so where u_il v_jl != 0 the step is the one fp32
+// subtract (or add) of d_l that the ordered deflation makes, rounded once,
+// and where u_il v_jl = 0 it adds a zero: x is unchanged (a -0 entry may turn
+// into +0, which no later sum, square or threshold can tell apart).  The
+// (weighted) row energies of the updated chunk are summed in fp64 on the way
+// out: lane partials over the sub-tiles, then across the warp.
+constexpr int kDefRows = 64;  // rows per CTA: 8 warps x 8 rows
+constexpr int kDefSub = 128;  // columns per sub-tile: 32 lanes x 4
+static_assert(kChunk % kDefSub == 0, "sub-tiles tile the chunk");
+constexpr size_t kDefSmem = sizeof(float2) * kMaxB * kDefRows + sizeof(float) * kMaxB * kDefSub;
+
+template <bool VEC>
+__global__ void __launch_bounds__(256, 3) deflate_kernel(float* __restrict__ R, int m, int n,
+                                                         const u64* __restrict__ Um,
+                                                         const u64* __restrict__ Us,
+                                                         const u64* __restrict__ Vm,
+                                                         const u64* __restrict__ Vs,
+                                                         const float* __restrict__ dblk, int bb,
+                                                         const float* __restrict__ w,
+                                                         double* __restrict__ rhop) {
+  extern __shared__ __align__(16) unsigned char dsm[];
+  float2* nd2 = (float2*)dsm;                                         // [kMaxB][kDefRows]
+  float* vf = (float*)(dsm + sizeof(float2) * kMaxB * kDefRows);      // [kMaxB][kDefSub]
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int i0 = blockIdx.x * kDefRows;
+  const int ch = blockIdx.y, j0 = ch * kChunk, j1 = min(n, j0 + kChunk);
   {
-    // kChunk / 256 = 4 entries per thread, all loads issued before the stores
-    u64 a[4], b[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int j = threadIdx.x + 256 * q;
-      a[q] = j < nj ? Vm[j0 + j] : 0ull;
-      b[q] = j < nj ? Vs[j0 + j] : 0ull;
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      vm[threadIdx.x + 256 * q] = a[q];
-      vs[threadIdx.x + 256 * q] = b[q];
+    const int r = tid & (kDefRows - 1), i = i0 + r;
+    const u64 um = i < m ? Um[i] : 0ull, us = i < m ? Us[i] : 0ull;
+    for (int l = tid / kDefRows; l < bb; l += 256 / kDefRows) {
+      float v = 0.f;
+      if ((um >> l) & 1ull) v = ((us >> l) & 1ull) ? dblk[l] : -dblk[l];
+      nd2[l * kDefRows + r] = make_float2(v, v);
     }
   }
-  if (threadIdx.x < kMaxB) d[threadIdx.x] = dblk[threadIdx.x];
-  __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int* ls = ls_s[wid];
-  float* dus = du_s[wid];
-  for (int rr = 0; rr < 2; ++rr) {
-    const int i = blockIdx.x * 16 + wid * 2 + rr;
-    if (i >= m) break;
-    const u64 um = Um[i];
-    if (um == 0ull) continue;  // untouched row: R and its energy partials stay
-    const u64 us = Us[i];
-    // active components in ascending order; nlo of them below 32
-    __syncwarp();
-    const int nl = __popcll(um), nlo = __popc((uint32_t)um);
-    if (lane == 0) {
-      int c = 0;
-      for (u64 bits = um; bits; bits &= bits - 1ull, ++c) {
-        const int l = __ffsll((long long)bits) - 1;
-        ls[c] = l;
-        dus[c] = ((us >> l) & 1ull) ? -d[l] : d[l];
+  const int r0 = 8 * wid;
+  double es[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) es[q] = 0.0;
+  for (int jt = j0; jt < j1; jt += kDefSub) {
+    __syncthreads();  // nd2 written; the previous sub-tile's codes no longer read
+    {
+      // thread -> column c, components l = tid / 128 + 2 t
+      const int c = tid & (kDefSub - 1), j = jt + c;
+      const u64 vm = j < j1 ? Vm[j] : 0ull, vs = j < j1 ? Vs[j] : 0ull;
+      for (int l = tid / kDefSub; l < bb; l += 256 / kDefSub) {
+        const uint32_t on = (uint32_t)(vm >> l) & 1u, neg = (uint32_t)(vs >> l) & 1u;
+        vf[l * kDefSub + c] = __uint_as_float(on ? (0x3f800000u | (neg << 31)) : 0u);
       }
     }
-    __syncwarp();
-    float* row = R + (size_t)i * n + j0;
-    double s = 0.0;
-    for (int jw = 0; jw < nj; jw += 128) {  // warp-uniform trip count (warp votes inside)
-      const int jb = jw + lane;
-      float x[4];
-      uint32_t plo[4], phi[4], nlo_[4], nhi[4];
-      bool any = false;
+    __syncthreads();
+    const int jc = jt + 4 * lane;
+    float2 x[8][2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = jb + 32 * e;
-        const bool ok = j < nj;
-        x[e] = ok ? row[j] : 0.f;
-        const u64 mm = ok ? vm[j] & um : 0ull, sg = ok ? vs[j] : 0ull;
-        const u64 P = mm & ~sg, N = mm & sg;
-        plo[e] = (uint32_t)P;
-        phi[e] = (uint32_t)(P >> 32);
-        nlo_[e] = (uint32_t)N;
-        nhi[e] = (uint32_t)(N >> 32);
-        any |= mm != 0ull;
-      }
-      if (__any_sync(0xffffffffu, any)) {
-        for (int t = 0; t < nlo; ++t) {  // components 0..31: same trip count on every lane
-          const uint32_t bit = 1u << ls[t];
-          const float du = dus[t];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (plo[e] & bit) x[e] = __fsub_rn(x[e], du);
-            if (nlo_[e] & bit) x[e] = __fadd_rn(x[e], du);
-          }
-        }
-        for (int t = nlo; t < nl; ++t) {  // components 32..63
-          const uint32_t bit = 1u << (ls[t] - 32);
-          const float du = dus[t];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (phi[e] & bit) x[e] = __fsub_rn(x[e], du);
-            if (nhi[e] & bit) x[e] = __fadd_rn(x[e], du);
-          }
+    for (int q = 0; q < 8; ++q) {
+      const int i = i0 + r0 + q;
+      const float* src = R + (size_t)(i < m ? i : 0) * n + jc;
+      float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < m) {
+        if (VEC) {
+          if (jc < j1) t = *(const float4*)src;
+        } else {
+          if (jc < j1) t.x = src[0];
+          if (jc + 1 < j1) t.y = src[1];
+          if (jc + 2 < j1) t.z = src[2];
+          if (jc + 3 < j1) t.w = src[3];
         }
       }
+      x[q][0] = make_float2(t.x, t.y);
+      x[q][1] = make_float2(t.z, t.w);
+    }
+#pragma unroll 2
+    for (int l = 0; l < bb; ++l) {
+      const float4 v = *(const float4*)(vf + l * kDefSub + 4 * lane);
+      const float2 v01 = make_float2(v.x, v.y), v23 = make_float2(v.z, v.w);
+      const float4* np = (const float4*)(nd2 + l * kDefRows + r0);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = jb + 32 * e;
-        if (j < nj) {
-          if ((plo[e] | phi[e] | nlo_[e] | nhi[e]) != 0u) row[j] = x[e];
-          const double wj = w ? (double)w[j0 + j] : 1.0;
-          s += wj * (double)x[e] * (double)x[e];
-        }
+      for (int q = 0; q < 4; ++q) {
+        const float4 a = np[q];  // {nd, nd} of rows r0 + 2q and r0 + 2q + 1
+        const float2 a0 = make_float2(a.x, a.y), a1 = make_float2(a.z, a.w);
+        x[2 * q][0] = __ffma2_rn(a0, v01, x[2 * q][0]);
+        x[2 * q][1] = __ffma2_rn(a0, v23, x[2 * q][1]);
+        x[2 * q + 1][0] = __ffma2_rn(a1, v01, x[2 * q + 1][0]);
+        x[2 * q + 1][1] = __ffma2_rn(a1, v23, x[2 * q + 1][1]);
       }
     }
-    s = warp_sum(s);
-    if (lane == 0) rhop[(size_t)ch * m + i] = s;
+    double wj[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) wj[e] = (jc + e < j1) ? (w ? (double)w[jc + e] : 1.0) : 0.0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int i = i0 + r0 + q;
+      if (i < m) {
+        float* dst = R + (size_t)i * n + jc;
+        const float xv[4] = {x[q][0].x, x[q][0].y, x[q][1].x, x[q][1].y};
+        if (VEC) {
+          if (jc < j1) *(float4*)dst = make_float4(xv[0], xv[1], xv[2], xv[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (jc + e < j1) dst[e] = xv[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) es[q] += wj[e] * (double)xv[e] * (double)xv[e];
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const double s = warp_sum(es[q]);
+    const int i = i0 + r0 + q;
+    if (lane == 0 && i < m) rhop[(size_t)ch * m + i] = s;
   }
 }
 
@@ -1000,7 +1082,10 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
   const size_t partsP = sk ? (size_t)planP.T * planP.S * 128 : (size_t)splitP * m;
   const size_t partsQ = sk ? (size_t)planQ.T * planQ.S * 128 : (size_t)splitQ * n;
   const int boundP = sk ? planP.S : splitP, boundQ = sk ? planQ.S : splitQ;
-  const int tgtU = (m + kTgtRows2 - 1) / kTgtRows2, tgtV = (n + kTgtRows2 - 1) / kTgtRows2;
+  // target CTAs: rows spread evenly over the SMs; rpart keeps 64-row CTAs
+  const int rpcU = target_rpc(m, nsm), rpcV = target_rpc(n, nsm);
+  const int tgtU = (m + rpcU - 1) / rpcU, tgtV = (n + rpcV - 1) / rpcV;
+  const int rpartV = (n + kRpartRows - 1) / kRpartRows;
   const int nch = (n + kChunk - 1) / kChunk;
   const int mx = std::max(m, n);
   const int Wm = (m + 31) / 32, Wn = (n + 31) / 32;
@@ -1021,12 +1106,12 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
   const size_t oQp = take(sizeof(float) * partsQ * b);
   const size_t oT = take(sizeof(double) * (size_t)mx * b);
   const size_t oCs = take(sizeof(double) * (size_t)std::max(tgtU, tgtV) * b);
-  const size_t oRp = take(sizeof(double) * (size_t)tgtV * b);
-  const size_t oQs = take(sizeof(double) * (size_t)n * b);
+  const size_t oRp = take(sizeof(double) * (size_t)rpartV * b);
   const size_t oThr = take(sizeof(double) * kMaxB);
+  const size_t oTick = take(sizeof(unsigned));
+  const size_t oQs = take(sizeof(double) * (size_t)n * b);
   const size_t oBopU = take((size_t)Wm * umma::kBBytes), oBopV = take((size_t)Wn * umma::kBBytes);
   const size_t oWpad = take(sizeof(float) * (size_t)Wn * 32);
-  const size_t oTick = take(sizeof(unsigned));
   const size_t oSV = take(sizeof(double) * b * b), oSU = take(sizeof(double) * b * b);
   const size_t oGU = take(sizeof(double) * b * b), oGV = take(sizeof(double) * b * b);
   const size_t oScal = take(sizeof(double) * 4);
@@ -1049,20 +1134,24 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
   double* T = (double*)(base + oT);
   double* Cs = (double*)(base + oCs);
   double* Rp = (double*)(base + oRp);
+  double* thr = (double*)(base + oThr);
+  unsigned* tick = (unsigned*)(base + oTick);
   double *SV = (double*)(base + oSV), *SU = (double*)(base + oSU);
   double *GU = (double*)(base + oGU), *GV = (double*)(base + oGV);
   double* scal = (double*)(base + oScal);
   float* dblk = (float*)(base + oD);
   int* bad = (int*)(base + oBad);
-  double* thr = (double*)(base + oThr);
   double* Qs = (double*)(base + oQs);
   unsigned char* BopU = (unsigned char*)(base + oBopU);
   unsigned char* BopV = (unsigned char*)(base + oBopV);
   float* wpad = (float*)(base + oWpad);
-  unsigned* tick = (unsigned*)(base + oTick);
   const double tau = (double)h.tau;
   int rc = EXTERND_OK;
   const TargetFn tgtP = target_for(boundP), tgtQ = target_for(boundQ);
+  cudaFuncSetAttribute(deflate_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)kDefSmem);
+  cudaFuncSetAttribute(deflate_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)kDefSmem);
   cudaFuncSetAttribute(tgtP, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgtSmem);
   cudaFuncSetAttribute(tgtQ, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTgtSmem);
   // the row-energy keys of the radix select stay in shared memory when they fit
@@ -1118,9 +1207,10 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
       tc_contract_rv(R, m, n, Vm, Vs, BopV, h.w, wpad, bb, sk ? &planP : nullptr, klenP, splitP,
                      Pp, h.wait_budget, st);
       cudaStreamWaitEvent(st, ev_join, 0);
-      tgtP<<<tgtU, 256, kTgtSmem, st>>>(Pp, splitP, m, bb, SV, tau, T, Cs, tick, thr, nullptr, sk,
-                                         planP.C, planP.U, planP.G, planP.S, stat, nullptr);
-      tern_kernel<<<(Wm * 32 + 63) / 64, 64, 0, st>>>(T, m, bb, thr, Um, Us, pB, Wm, BopU);
+      tgtP<<<tgtU, kTgtThreads, kTgtSmem, st>>>(Pp, splitP, m, rpcU, bb, SV, tau, T, Cs, tick,
+                                                 thr, nullptr, sk, planP.C, planP.U, planP.G,
+                                                 planP.S, stat, nullptr);
+      tern_kernel<<<Wm, 256, 0, st>>>(T, m, bb, thr, Um, Us, pB, Wm, BopU);
       cudaEventRecord(ev_fork, st);
       cudaStreamWaitEvent(side, ev_fork, 0);
       gram_kernel<<<gblocks, gthreads, 0, side>>>(pB, Wm, bb, nullptr, GU);
@@ -1129,10 +1219,11 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
       tc_contract_rtu(R, m, n, Um, Us, BopU, bb, sk ? &planQ : nullptr, klenQ, splitQ, Qp,
                       h.wait_budget, st);
       cudaStreamWaitEvent(st, ev_join, 0);
-      tgtQ<<<tgtV, 256, kTgtSmem, st>>>(Qp, splitQ, n, bb, SU, tau, T, Cs, tick, thr,
-                                         it == h.iters - 1 ? Qs : nullptr, sk, planQ.C, planQ.U,
-                                         planQ.G, planQ.S, stat, naive_w);
-      tern_kernel<<<(Wn * 32 + 63) / 64, 64, 0, st>>>(T, n, bb, thr, Vm, Vs, pC, Wn, BopV);
+      tgtQ<<<tgtV, kTgtThreads, kTgtSmem, st>>>(Qp, splitQ, n, rpcV, bb, SU, tau, T, Cs, tick,
+                                                 thr, it == h.iters - 1 ? Qs : nullptr, sk,
+                                                 planQ.C, planQ.U, planQ.G, planQ.S, stat,
+                                                 naive_w);
+      tern_kernel<<<Wn, 256, 0, st>>>(T, n, bb, thr, Vm, Vs, pC, Wn, BopV);
       if (tr) {
         u64* at = tr + 2 * (size_t)n + (size_t)it * 2 * ((size_t)m + n);
         record(at, Um, Us, m);
@@ -1140,9 +1231,14 @@ static int block_enqueue(const BlockHostArgs& h, cudaStream_t st, cudaStream_t s
       }
     }
     gram_kernel<<<gblocks, gthreads, 0, st>>>(pC, Wn, bb, h.w, GV);
-    rpart_kernel<<<tgtV, 256, 0, st>>>(Qs, n, bb, Vm, Vs, h.w, Rp);
-    dsolve_kernel<<<1, 256, 0, st>>>(GU, GV, Rp, tgtV, bb, scal, c0, h.D, h.energy, dblk);
-    deflate_kernel<<<dim3((m + 15) / 16, nch), 256, 0, st>>>(R, m, n, Um, Us, Vm, Vs, dblk, h.w, rhop);
+    rpart_kernel<<<rpartV, 256, 0, st>>>(Qs, n, bb, Vm, Vs, h.w, Rp);
+    dsolve_kernel<<<1, 256, 0, st>>>(GU, GV, Rp, rpartV, bb, scal, c0, h.D, h.energy, dblk);
+    if (n % 4 == 0)
+      deflate_kernel<true><<<dim3((m + kDefRows - 1) / kDefRows, nch), 256, kDefSmem, st>>>(
+          R, m, n, Um, Us, Vm, Vs, dblk, bb, h.w, rhop);
+    else
+      deflate_kernel<false><<<dim3((m + kDefRows - 1) / kDefRows, nch), 256, kDefSmem, st>>>(
+          R, m, n, Um, Us, Vm, Vs, dblk, bb, h.w, rhop);
     chk();
   }
   int* status = status_word_ptr();

@@ -378,9 +378,14 @@ __global__ void __launch_bounds__(kThreads, 1) contract_kernel(
       for (int t = 0; t < 32; ++t)
         if (chalf * 32 + t < bb) Xp[((size_t)split * M + gi) * bb + chalf * 32 + t] = 0.f;
   }
+  // every warp's tensor-memory loads are complete (tcgen05.wait::ld) and
+  // ordered before the barrier; the deallocating warp orders itself after it
   tc_fence_before();
   __syncthreads();
-  if (wid == 0) tmem_dealloc(tmem, kN);
+  if (wid == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kN);
+  }
 }
 
 
