@@ -7,7 +7,8 @@ iterations, block = 1) through the C ABI.  Prints one JSON line on rank 0.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload attn2560|mlp9728_b64|mlp9728_b1|block_layer]
-  python bench.py --case attn2560_k64|mlp9728_3blocks|apply_attn2560   (small profiling cases)
+  python bench.py --case attn2560_k64|attn2560_phases|mlp9728_3blocks|apply_attn2560
+                                                   (small profiling and breakdown cases)
 
 --workload picks another configuration (default: the 2560 x 2560 one above);
 mlp9728_b64 / _b1 decompose the 9728 x 2560 MLP-shaped matrix (mu = 2) with
@@ -475,6 +476,34 @@ def run_case(args):
     elif args.case == "mlp9728_3blocks":
         wl = W.config_mlp9728(64)
         mu, block = 3 * 64 / min(wl.m, wl.n), 64
+    elif args.case == "attn2560_phases":
+        # where one component's time goes: SM cycles of CTA 0 per phase, from
+        # the traced entry point's counters, over 512 components of the
+        # benchmark matrix (the same kernel and launch plan as the benchmark)
+        wl = W.config_attn2560()
+        A = torch.from_numpy(wl.a).cuda()
+        mu = 512 / min(wl.m, wl.n)
+        X.decompose_traced(A, mu, wl.tau, wl.iters, [])
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        f, tr, st = X.decompose_traced(A, mu, wl.tau, wl.iters, [])
+        ev1.record()
+        ev1.synchronize()
+        s = tr.stats.cpu().numpy()
+        names = ["setup", "R W v pass", "cluster gather of y", "y exchange and u threshold",
+                 "R^T u pass", "z exchange", "z cluster step", "scale and emit", "deflation",
+                 "statistics exchange"]
+        us = ev0.elapsed_time(ev1) * 1000.0 / f.k
+        cyc = s[6:16].astype(float)
+        clk = cyc.sum() / (us * f.k)  # cycles per microsecond over the launch
+        print(json.dumps({"case": args.case, "components": f.k, "plan": {"clusters": int(s[2]),
+                          "cta_per_cluster": int(s[3]), "smem_rows": int(s[4]), "rows": int(s[5])},
+                          "us_per_component": us, "sm_mhz": clk,
+                          "us_per_component_by_phase": {nm: c / clk / f.k for nm, c in zip(names, cyc)},
+                          "status": st}))
+        if st != X.OK:
+            raise SystemExit(1)
+        return
     elif args.case == "apply_attn2560":
         # the inference kernel on the benchmark matrix's factors (mu = 3): the
         # decomposition, then three one-vector calls
@@ -510,8 +539,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", choices=WORKLOADS, default="attn2560")
-    ap.add_argument("--case", choices=("attn2560_k64", "mlp9728_3blocks", "apply_attn2560"),
-                    default=None)
+    ap.add_argument("--case", choices=("attn2560_k64", "attn2560_phases", "mlp9728_3blocks",
+                                       "apply_attn2560"), default=None)
     args = ap.parse_args()
     if args.case:
         run_case(args)
