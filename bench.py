@@ -181,6 +181,28 @@ def _profiled_traffic(kernel: str, workload: str):
         return None
 
 
+def _sweep_report(X, wl, dev, sweeps=2):
+    """Refinement sweeps on the step's matrix (outside the timed region): the
+    energy after the greedy pass and after each sweep, the gain of each sweep
+    in energy points, and the device time of the whole call."""
+    import torch
+    A = torch.from_numpy(wl.a).to(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    f = X.decompose(A, wl.mu, wl.tau, wl.iters, sweeps=sweeps)
+    ev1.record()
+    ev1.synchronize()
+    e0 = float(f.energy[-1])
+    es = [float(e) for e in f.sweep_energy[:sweeps].cpu()]
+    prev, gains = e0, []
+    for e in es:
+        gains.append(100.0 * (e - prev))
+        prev = e
+    return {"sweeps": sweeps, "energy_after_greedy_pct": 100.0 * e0,
+            "energy_after_sweep_pct": [100.0 * e for e in es], "gain_points": gains,
+            "ms_greedy_plus_sweeps": ev0.elapsed_time(ev1)}
+
+
 def _host_cpu():
     model = None
     try:
@@ -439,6 +461,8 @@ def run_ours(args, rank, world, local_rank):
             # the rank this matrix needs for Q4_K's per-matrix energy (99.4%,
             # Pith review), read off the run's energy trace on the device
             cfg["rank_for_99.4pct_energy"] = X.rank_for_energy(outs[0].energy, 0.994)
+            if world == 1 and not args.no_sweeps:
+                cfg["refinement_sweeps"] = _sweep_report(X, wls[0], dev)
     else:
         cfg["energy_preserved_pct"] = {wl.name: 100.0 * e for wl, e in zip(wls, energies)}
         cfg["factors"] = {wl.name: r for wl, r in zip(wls, reports)}
@@ -538,6 +562,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the refinement-sweep report (a greedy pass plus two sweeps)")
     ap.add_argument("--workload", choices=WORKLOADS, default="attn2560")
     ap.add_argument("--case", choices=("attn2560_k64", "attn2560_phases", "mlp9728_3blocks",
                                        "apply_attn2560"), default=None)

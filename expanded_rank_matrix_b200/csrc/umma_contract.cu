@@ -433,6 +433,10 @@ constexpr int kConvGroups = 2;                          // converter groups, alt
 constexpr int kThreadsP = 32 * kConvWarp0 + 256 * kConvGroups;
 constexpr int kSmemP = kS32 * kStageBytesP + 1024;
 static_assert(kAstage0 + kS32 * kAcolsStage <= kTmemCols, "tensor memory budget");
+// A converter group waits on stage s's `full` barrier by phase parity; that is
+// unambiguous only if the same group consumed the stage's previous fill (chunk
+// i - kS32) and so saw it land: every group must own whole stages.
+static_assert(kS32 % kConvGroups == 0, "converter groups own whole ring stages");
 static_assert(kStageBytesP % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(2 * (kSmemP + 1024) > 228 * 1024, "the ring must keep the kernel at one CTA per SM");
 static_assert(kSmemP <= 227 * 1024, "shared memory per CTA");
