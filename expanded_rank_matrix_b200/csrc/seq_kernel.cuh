@@ -728,9 +728,11 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
     double* rsa = (double*)zred;  // [NC][CS] slice sums of squares (one-round path)
     const bool one_round = !with_row || (a.NC <= 16 && TC + a.NC <= kThreads &&
                                          2 * a.NC * CS <= L.zred_floats);
-    // the CTAs' slice statistics: a thread each when the block has enough
-    // threads, else the record threads fetch their cluster's as well
-    const bool rsa_own = TC + a.NC + a.NC * CS <= kThreads;
+    // the CTAs' slice statistics: fetched by the threads past the record
+    // range, each taking every nspare-th one (a few waits at most); only if
+    // no thread is spare do the record threads fetch their cluster's
+    const int rs0 = TC + a.NC, nspare = kThreads - rs0;
+    const bool rsa_spare = nspare > 0;
     const long long cstride = (long long)CS * a.recw;
     const int rbase = (with_row && one_round) ? TC : 0;  // first thread of the record range
     uint32_t slice[16];
@@ -745,18 +747,19 @@ __global__ void __launch_bounds__(kThreads, 1) seq_als_kernel(const SeqArgs a) {
       x_bv[cc] = u2f(p[5]);
       x_r2[cc] = u2d(p[6], p[7]);
       x_bad[cc] = p[8];
-      if (with_row && one_round && !rsa_own)
+      if (with_row && one_round && !rsa_spare)
         for (int qq = 0; qq < CS; ++qq) {
           uint32_t p2[2];
           xw_wait_n<2>(rec(s, cc, qq) + TCp, 1, 2, ep, p2, ab, a.budget, a.abort_word);
           rsa[cc * CS + qq] = u2d(p2[0], p2[1]);
         }
-    } else if (with_row && one_round && rsa_own && tid >= TC + a.NC &&
-               tid < TC + a.NC + a.NC * CS) {
-      const int t = tid - TC - a.NC, cc = t / CS, qq = t - cc * CS;
-      uint32_t p[2];
-      xw_wait_n<2>(rec(s, cc, qq) + TCp, 1, 2, ep, p, ab, a.budget, a.abort_word);
-      rsa[t] = u2d(p[0], p[1]);
+    } else if (with_row && one_round && rsa_spare && tid >= rs0) {
+      for (int t = tid - rs0; t < a.NC * CS; t += nspare) {
+        const int cc = t / CS, qq = t - cc * CS;
+        uint32_t p[2];
+        xw_wait_n<2>(rec(s, cc, qq) + TCp, 1, 2, ep, p, ab, a.budget, a.abort_word);
+        rsa[t] = u2d(p[0], p[1]);
+      }
     } else if (with_row && one_round && tid < TC) {
       xw_wait_n<16>(rec(s, 0, q) + tid, cstride, a.NC, ep, slice, ab, a.budget, a.abort_word);
     }
