@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(256, 1) inv_kernel(const double* __restrict__ 
 // The rows are split evenly over at most one CTA per SM: CTA c takes rows
 // [c rpc, (c+1) rpc) with rpc <= 80, so no SM holds twice the work of
 // another.  The split-K / stream-K partials are summed (in partial order,
-// fp64) into a transposed tile Xt[l2][row] in shared memory next to S -- each
+// fp64) into a row-major tile Xs[row][l2] in shared memory next to S -- each
 // thread loads 4 consecutive columns of 4 rows, float4 per partial, all
 // partials in flight (NS >= partials is a compile-time bound).  Thread
 // (rg, cg) then forms the 4 x 4 block rows 4rg.., columns 4cg.. of T: 16
@@ -528,7 +528,9 @@ constexpr int kTgtMaxRows = 80;      // rows per CTA at most (20 groups x 4)
 constexpr int kTgtRedGroups = kTgtThreads / kMaxB;  // 5 summing groups in the last CTA
 constexpr int kTgtRedLoads = 32;     // loads in flight per thread in the last CTA
 constexpr int kMaxSplits = kMaxSegs;  // partials per output row (split-K or stream-K)
-constexpr int kXs = kTgtMaxRows + 2;  // padded row of the transposed tile (16-byte aligned)
+// padded row of the X tile: even (16-byte aligned pairs), and 4 rows apart
+// land 16 banks apart, so the two row groups a warp reads never collide
+constexpr int kXs = kMaxB + 2;
 // rows per CTA for `rows` rows on nsm SMs
 inline int target_rpc(int rows, int nsm) {
   const int r = (rows + nsm - 1) / std::max(nsm, 1);
@@ -546,11 +548,18 @@ __global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
     const float* __restrict__ wsc) {
   extern __shared__ __align__(16) double tsh[];
   double* Ss = tsh;                                                    // [64][64]: S[l2][l]
-  double* Xt = tsh + kMaxB * kMaxB;                                    // [64][kXs]
-  double (*part)[kMaxB] = (double (*)[kMaxB])(Xt + kMaxB * kXs);       // [20][64]
+  double* Xt = tsh + kMaxB * kMaxB;                                    // [80][kXs]
+  double (*part)[kMaxB] = (double (*)[kMaxB])(Xt + kTgtMaxRows * kXs);  // [20][64]
   __shared__ bool last;
+  __shared__ int np_s[2];  // partials of the CTA's first and last 128-row tile
   const int tid = threadIdx.x;
   const int x0 = blockIdx.x * rpc, nr = min(rpc, rows - x0);
+  if (tid < 2) {
+    // the CTA's rows (at most 80) meet at most two tiles; the segment count
+    // costs 64-bit divisions, so it is found once per tile, not per row
+    const int xt = tid == 0 ? x0 : x0 + nr - 1;
+    np_s[tid] = sk ? umma::sk_nseg(xt / umma::kM, C, U, G) : splits;
+  }
   {
     constexpr int kSL = (kMaxB * kMaxB + kTgtThreads - 1) / kTgtThreads;
     double sv[kSL];
@@ -565,6 +574,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
       if (p < kMaxB * kMaxB) Ss[p] = sv[q];
     }
   }
+  __syncthreads();  // np_s
   {
     // thread: columns lq .. lq+3 (lq = 4 (tid % 16)), rows tid / 16 + 20 h
     const int lq = (tid & 15) * 4, rr = tid >> 4;
@@ -580,7 +590,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
         const int r = rr + 20 * (h0 + h), x = x0 + r;
         const bool ok = r < nr && lq < bb;
         const int xs = ok ? x : 0;
-        np[h] = sk ? umma::sk_nseg(xs / umma::kM, C, U, G) : splits;
+        np[h] = ok ? np_s[(xs / umma::kM) != (x0 / umma::kM)] : 0;
         const size_t prow = sk ? ((size_t)(xs / umma::kM) * Sslots * umma::kM + xs % umma::kM)
                                : (size_t)xs;
         const float* src = Xp + prow * bb + (ok ? lq : 0);
@@ -613,10 +623,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
             s3 += (double)v[h][sp].w;
           }
         const int r = rr + 20 * (h0 + h);
-        Xt[(lq + 0) * kXs + r] = s0;
-        Xt[(lq + 1) * kXs + r] = s1;
-        Xt[(lq + 2) * kXs + r] = s2;
-        Xt[(lq + 3) * kXs + r] = s3;
+        *(double2*)(Xt + r * kXs + lq) = make_double2(s0, s1);
+        *(double2*)(Xt + r * kXs + lq + 2) = make_double2(s2, s3);
         const int x = x0 + r;
         if (Xout && r < nr) {
           const double sx[4] = {s0, s1, s2, s3};
@@ -635,17 +643,25 @@ __global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
   if (4 * rg < nr) {
+    // two l2 per step (X entries past bb and S rows past bb are zero)
+    const double* xr = Xt + (4 * rg) * kXs;
 #pragma unroll 2
-    for (int l2 = 0; l2 < bb; ++l2) {
-      const double2 xa = *(const double2*)(Xt + l2 * kXs + 4 * rg);
-      const double2 xb = *(const double2*)(Xt + l2 * kXs + 4 * rg + 2);
-      const double2 sa = *(const double2*)(Ss + l2 * kMaxB + 4 * cg);
-      const double2 sb = *(const double2*)(Ss + l2 * kMaxB + 4 * cg + 2);
-      const double xv[4] = {xa.x, xa.y, xb.x, xb.y}, svv[4] = {sa.x, sa.y, sb.x, sb.y};
+    for (int l2 = 0; l2 < bb; l2 += 2) {
+      double2 xp[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) xp[i] = *(const double2*)(xr + i * kXs + l2);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] += xv[i] * svv[j];
+      for (int h = 0; h < 2; ++h) {
+        const double2 sa = *(const double2*)(Ss + (l2 + h) * kMaxB + 4 * cg);
+        const double2 sb = *(const double2*)(Ss + (l2 + h) * kMaxB + 4 * cg + 2);
+        const double svv[4] = {sa.x, sa.y, sb.x, sb.y};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const double xv = h ? xp[i].y : xp[i].x;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] += xv * svv[j];
+        }
+      }
     }
   }
   double cs[4] = {0.0, 0.0, 0.0, 0.0};
@@ -715,7 +731,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1) target_kernel(
   if (tid == 0) *ticket = 0u;
 }
 constexpr size_t kTgtSmem =
-    sizeof(double) * (kMaxB * kMaxB + kMaxB * kXs + (kTgtThreads / 16) * kMaxB);
+    sizeof(double) * (kMaxB * kMaxB + kTgtMaxRows * kXs + (kTgtThreads / 16) * kMaxB);
 // the target kernel instantiated for a partial-count bound
 typedef void (*TargetFn)(const float*, int, int, int, int, const double*, double, double*,
                          double*, unsigned*, double*, double*, int, int, long long, int, int, int,
