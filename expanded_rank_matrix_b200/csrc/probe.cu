@@ -1,8 +1,8 @@
 // Read-bandwidth probes for the on-chip rooflines: shared memory (every SM
 // streams its own shared memory) and L2 (every SM streams an L2-resident
 // buffer).  The sequential kernel keeps the residual in shared memory and
-// the block path's operands mostly in L2, so their kernels are judged
-// against these rates as well as against HBM.
+// the block path's operands mostly in L2, so their kernels are compared
+// with these rates as well as with HBM.
 
 #include <cuda_runtime.h>
 
